@@ -1,0 +1,968 @@
+// Device code of libamk (sm_100a): the persistent decode kernel, its routines, and the weight packer.
+//
+// One CTA per SM, 17 warps: warp 16 is the producer, whose elected lane streams every byte this CTA
+// will read (weight rows of its GEMV tasks, KV rows of its attention chunk) into a 6 x 32 KB
+// shared-memory ring with cp.async.bulk, completion tracked by one mbarrier per slot. The producer
+// never waits on other CTAs, so the next tasks' weights arrive while the compute warps wait on a
+// counter: this is the "prefetch the next layer's weights while the current layer computes" of
+// "AutoMegaKernel: A Statically-Checked Agent Harness for Self-Retargeting Megakernel Synthesis"
+// (README summary), with dependencies carried by counters instead of grid barriers (technical
+// summary, "Methodology", Layer 0: wait -> dispatch -> signal on monotonic counters).
+//
+// Warps 0..15 compute. Every wait is bounded by a %globaltimer deadline; when one expires the CTA
+// raises a device abort flag plus a host-visible status word and every later counter wait returns
+// at once, so the launch always completes (outputs are then garbage and the handle reports it).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "amk_internal.h"
+
+namespace amk {
+namespace dev {
+
+// ------------------------------------------------------------------------------------------------
+// PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.volatile.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// acc0 += lo(w) * lo(a); acc1 += hi(w) * hi(a)   (f16 x f16 -> f32, one rounding each)
+__device__ __forceinline__ void fma2_f16_f32(float& acc0, float& acc1, uint32_t w, uint32_t a) {
+  asm("{\n\t.reg .f16 w0, w1, a0, a1;\n\t"
+      "mov.b32 {w0, w1}, %2;\n\t"
+      "mov.b32 {a0, a1}, %3;\n\t"
+      "fma.rn.f32.f16 %0, w0, a0, %0;\n\t"
+      "fma.rn.f32.f16 %1, w1, a1, %1;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(w), "r"(a));
+}
+// acc += {lo, hi} * {a0, a1} with one packed fp32 FMA
+__device__ __forceinline__ void ffma2(unsigned long long& acc, float lo, float hi, float a0, float a1) {
+  asm("{\n\t.reg .b64 wv, av;\n\t"
+      "mov.b64 wv, {%1, %2};\n\t"
+      "mov.b64 av, {%3, %4};\n\t"
+      "fma.rn.f32x2 %0, wv, av, %0;\n\t}"
+      : "+l"(acc)
+      : "f"(lo), "f"(hi), "f"(a0), "f"(a1));
+}
+__device__ __forceinline__ float f2sum(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Shared memory
+
+struct Misc {
+  int token;
+  int flag;
+  float red[kConsumerWarps];
+  float am_v[kConsumerWarps];
+  int am_i[kConsumerWarps];
+  float lm_v;
+  int lm_i;
+};
+static_assert(sizeof(Misc) + 2 * kSlots * 8 <= kMiscBytes, "misc region");
+
+struct Smem {
+  uint8_t* ring;
+  float* part;
+  float* aux;
+  float* scale;
+  uint64_t* full;
+  uint64_t* empty;
+  Misc* misc;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* base) {
+  Smem s;
+  s.ring = base;
+  s.part = reinterpret_cast<float*>(base + kRingBytes);
+  s.aux = reinterpret_cast<float*>(base + kRingBytes + kPartBytes);
+  s.scale = reinterpret_cast<float*>(base + kRingBytes + kPartBytes + kAuxBytes);
+  uint8_t* m = base + kRingBytes + kPartBytes + kAuxBytes + kScaleBytes;
+  s.full = reinterpret_cast<uint64_t*>(m);
+  s.empty = s.full + kSlots;
+  s.misc = reinterpret_cast<Misc*>(m + 2 * kSlots * 8);
+  return s;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Failure handling and waits
+
+__device__ void raise_abort(const Params& p, uint32_t detail) {
+  if (atomicCAS(p.abort_flag, 0u, 1u) == 0u) {
+    *p.status = 0x80000000u | detail;
+    __threadfence_system();
+  }
+}
+
+// Thread 0 of the compute warps spins until counter >= target (mod 2^32), bounded by the timeout.
+// Returns false if the wait expired or another CTA aborted (the caller then carries on: data are
+// garbage but every thread keeps the same control flow, so the launch still completes).
+__device__ bool spin_counter(const Params& p, int ctr, uint32_t target) {
+  const uint32_t* c = p.ctr + ctr;
+  if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
+  if (ld_volatile(p.abort_flag)) return false;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(20);
+    if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
+    if ((it & 15) == 0) {
+      if (ld_volatile(p.abort_flag)) return false;
+      if (globaltimer() - t0 > p.timeout_ns) {
+        raise_abort(p, (1u << 16) | (uint32_t)ctr);
+        return false;
+      }
+    }
+  }
+}
+
+// All compute threads call this; thread 0 waits, then the compute barrier publishes it.
+__device__ __forceinline__ void wait_counter(const Params& p, int ctr, uint32_t mult) {
+  if (threadIdx.x == 0) spin_counter(p, ctr, p.epoch * mult);
+  bar_compute();
+}
+
+__device__ __forceinline__ void signal_counter(const Params& p, int ctr) {
+  // caller has passed a compute barrier after the task's last global store
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(p.ctr + ctr, 1u);
+  }
+}
+
+// Bounded wait on a ring mbarrier phase. Its bound is 4x the counter bound, so a stalled counter is
+// always reported first (the ring drains once the counter waits give up); this one only expires if
+// the copy protocol itself broke.
+__device__ __forceinline__ void wait_slot(const Params& p, uint64_t* bar, uint32_t parity, uint32_t detail) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > 4 * p.timeout_ns) {
+      raise_abort(p, detail);
+      return;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Byte stream of one task (shared by the producer and the compute warps so both walk the same
+// sequence of ring slots).
+
+__device__ __forceinline__ const void* gemv_weights(const Params& p, int op, int l) {
+  switch (op) {
+    case OP_QKV: return p.layers[l].wqkv;
+    case OP_O: return p.layers[l].wo;
+    case OP_GU: return p.layers[l].wgu;
+    case OP_DOWN: return p.layers[l].wdown;
+    default: return p.lm_w;
+  }
+}
+__device__ __forceinline__ const uint16_t* gemv_scales(const Params& p, int op, int l) {
+  switch (op) {
+    case OP_QKV: return p.layers[l].sqkv;
+    case OP_O: return p.layers[l].so;
+    case OP_GU: return p.layers[l].sgu;
+    case OP_DOWN: return p.layers[l].sdown;
+    default: return p.lm_s;
+  }
+}
+__device__ __forceinline__ bool is_gemv(int op) { return op == OP_QKV || op == OP_O || op == OP_GU || op == OP_DOWN || op == OP_LM; }
+
+// ------------------------------------------------------------------------------------------------
+// Producer
+
+__device__ void producer(const Params& p, const Task* tasks, int nt, Smem& s) {
+  const uint64_t pol = policy_evict_first();
+  uint32_t it = 0;
+  auto acquire_slot = [&](uint32_t i) -> int {
+    const int slot = i % kSlots;
+    if (i >= (uint32_t)kSlots) wait_slot(p, &s.empty[slot], ((i / kSlots) - 1) & 1, (3u << 16) | slot);
+    return slot;
+  };
+  for (int ti = 0; ti < nt; ++ti) {
+    const Task t = tasks[ti];
+    if (is_gemv(t.op)) {
+      const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
+      const uint8_t* w = static_cast<const uint8_t*>(gemv_weights(p, t.op, t.layer));
+      for (int r = 0; r < t.b; r += g.rs, ++it) {
+        const int n = min(g.rs, t.b - r);
+        const int slot = acquire_slot(it);
+        const uint32_t bytes = (uint32_t)n * (uint32_t)g.rb;
+        mbar_expect_tx(&s.full[slot], bytes);
+        bulk_g2s(s.ring + slot * kSlotBytes, w + (size_t)(t.a + r) * g.rb, bytes, &s.full[slot], pol);
+      }
+    } else if (t.op == OP_ATTN) {
+      const int P = p.pos + 1;
+      const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
+      if (t.b >= C) continue;
+      int cb, ce;
+      attn_chunk_range(P, C, t.b, &cb, &ce);
+      const int nps = attn_positions_per_slot(p.hd);
+      const size_t row_bytes = (size_t)p.hd * 2;
+      const size_t head_off = ((size_t)t.layer * p.Hkv + t.a) * p.max_seq;
+      for (int blk = cb; blk < ce; blk += nps, ++it) {
+        const int be = min(blk + nps, ce);
+        const int ntma = min(be, p.pos) - blk;   // row `pos` is written this step: patched in smem
+        const int slot = acquire_slot(it);
+        if (ntma > 0) {
+          const uint32_t bytes = (uint32_t)(ntma * row_bytes);
+          mbar_expect_tx(&s.full[slot], 2 * bytes);
+          uint8_t* dst = s.ring + slot * kSlotBytes;
+          bulk_g2s(dst, p.kcache + (head_off + blk) * p.hd, bytes, &s.full[slot], pol);
+          bulk_g2s(dst + kSlotBytes / 2, p.vcache + (head_off + blk) * p.hd, bytes, &s.full[slot], pol);
+        } else {
+          mbar_arrive(&s.full[slot]);
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// GEMV
+
+// Block-wide sum over the compute threads in a fixed order (deterministic).
+__device__ float block_sum(float v, Smem& s) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) s.misc->red[warp] = v;
+  bar_compute();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) t += s.misc->red[w];
+  bar_compute();
+  return t;
+}
+
+// Sum of 4 per-lane values for 4 rows over the warp; lanes with (lane & 7) == 0 return row
+// (lane >> 3) & 3's total (transposed butterfly: 6 shuffles for 4 rows).
+__device__ __forceinline__ float reduce4_rows(float a0, float a1, float a2, float a3) {
+  const int lane = threadIdx.x & 31;
+  const bool u16 = lane & 16;
+  float k0 = u16 ? a2 : a0, t0 = u16 ? a0 : a2;
+  float k1 = u16 ? a3 : a1, t1 = u16 ? a1 : a3;
+  k0 += __shfl_xor_sync(0xffffffffu, t0, 16);
+  k1 += __shfl_xor_sync(0xffffffffu, t1, 16);
+  const bool u8 = lane & 8;
+  float u = u8 ? k1 : k0, v = u8 ? k0 : k1;
+  u += __shfl_xor_sync(0xffffffffu, v, 8);
+  u += __shfl_xor_sync(0xffffffffu, u, 4);
+  u += __shfl_xor_sync(0xffffffffu, u, 2);
+  u += __shfl_xor_sync(0xffffffffu, u, 1);
+  return u;
+}
+
+template <int GB>
+struct GroupWords { static constexpr int N = GB >= 4 ? GB / 4 : 1; };
+
+template <int GB>
+__device__ __forceinline__ void lds_group(const uint8_t* ptr, uint32_t (&w)[GroupWords<GB>::N]) {
+  if constexpr (GB == 16) {
+    uint4 v = *reinterpret_cast<const uint4*>(ptr);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (GB == 8) {
+    uint2 v = *reinterpret_cast<const uint2*>(ptr);
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (GB == 4) {
+    w[0] = *reinterpret_cast<const uint32_t*>(ptr);
+  } else {
+    w[0] = *reinterpret_cast<const uint16_t*>(ptr);
+  }
+}
+
+// int8 group against f16 activations: acc += sum_e (q_e + 1152) * a_e  (the +1152 is removed later
+// with the thread's activation sum). Each int8 byte becomes the f16 1024 + (q ^ 0x80) exactly.
+template <int GB>
+__device__ __forceinline__ void dot_i8(float& acc0, float& acc1, const uint32_t (&w)[GroupWords<GB>::N],
+                                       const uint32_t* a) {
+  if constexpr (GB >= 4) {
+#pragma unroll
+    for (int k = 0; k < GB / 4; ++k) {
+      const uint32_t x = w[k] ^ 0x80808080u;
+      const uint32_t h01 = __byte_perm(x, 0x64646464u, 0x4140);
+      const uint32_t h23 = __byte_perm(x, 0x64646464u, 0x4342);
+      fma2_f16_f32(acc0, acc1, h01, a[2 * k]);
+      fma2_f16_f32(acc0, acc1, h23, a[2 * k + 1]);
+    }
+  } else {
+    const uint32_t x = w[0] ^ 0x8080u;
+    const uint32_t h01 = __byte_perm(x, 0x64646464u, 0x4140);
+    fma2_f16_f32(acc0, acc1, h01, a[0]);
+  }
+}
+
+// bf16 group against fp32 activations (packed fp32 FMAs).
+template <int GB>
+__device__ __forceinline__ void dot_bf16(unsigned long long& acc, const uint32_t (&w)[GroupWords<GB>::N],
+                                         const float* a) {
+#pragma unroll
+  for (int k = 0; k < GB / 4; ++k) {
+    const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xffff0000u);
+    ffma2(acc, lo, hi, a[2 * k], a[2 * k + 1]);
+  }
+}
+
+// Source vector element `e` of the GEMV of `op` (before the f16 / fp32 packing).
+struct VecSrc {
+  const float* f32;       // x / attn_out / act, or null
+  const uint16_t* bf16;   // embedding row (first QKV), or null
+  const uint16_t* gain;   // RMSNorm gain, or null
+  float inv;              // 1 / rms, or 1
+};
+
+__device__ __forceinline__ float vec_elem(const VecSrc& v, int e) {
+  float x = v.f32 ? __ldcg(v.f32 + e) : bf2f(v.bf16[e]);
+  if (v.gain) x = x * v.inv * bf2f(v.gain[e]);
+  return x;
+}
+
+template <bool I8, int GB>
+__device__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it, int token) {
+  constexpr int NRMAX = (I8 ? 32 : 64) / GB;             // 16 f16x2 or 32 fp32 activation registers
+  constexpr int EPG = I8 ? GB : GB / 2;                 // elements per group
+  constexpr int AW = I8 ? (GB >= 4 ? GB / 2 : 1) : EPG; // activation registers per group
+  const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int op = t.op, l = t.layer, row0 = t.a, nrows = t.b;
+  const bool first = t.flags & kFirstOfStage;
+
+  const uint16_t* sc = I8 ? gemv_scales(p, op, l) : nullptr;
+  if (I8 && sc)
+    for (int i = tid; i < nrows; i += kConsumerThreads) s.scale[i] = bf2f(__ldg(sc + row0 + i));
+
+  if (p.sync && first && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
+
+  // ---- activations of this thread's groups (kept in registers for the whole task) ----
+  VecSrc v{nullptr, nullptr, nullptr, 1.f};
+  if (op == OP_QKV || op == OP_GU || op == OP_LM) {
+    if (op == OP_QKV && l == 0) v.bf16 = p.embed + (size_t)token * p.d;
+    else v.f32 = p.x;
+    v.gain = op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : p.final_norm;
+    float ss = 0.f;
+    for (int e = tid; e < p.d; e += kConsumerThreads) {
+      const float x = v.f32 ? __ldcg(v.f32 + e) : bf2f(v.bf16[e]);
+      ss += x * x;
+    }
+    ss = block_sum(ss, s);
+    v.inv = rsqrtf(ss / (float)p.d + p.eps);
+  } else {
+    v.f32 = op == OP_O ? p.attn_out : p.act;
+  }
+
+  const int rp = warp / g.wpg, wg = warp % g.wpg;
+  const bool active = rp < g.rp;
+  uint32_t ah[I8 ? NRMAX * AW : 1];
+  float af[I8 ? 1 : NRMAX * AW];
+  float asum = 0.f;
+#pragma unroll
+  for (int j = 0; j < NRMAX; ++j) {
+    const int col = j * g.wpg + wg;
+    const bool ok = active && j < g.nr && col < g.wg_total;
+    const int e0 = (col * 32 + lane) * EPG;
+    if constexpr (I8) {
+#pragma unroll
+      for (int k = 0; k < AW; ++k) {
+        float x0 = 0.f, x1 = 0.f;
+        if (ok) {
+          x0 = vec_elem(v, e0 + 2 * k);
+          if (EPG > 1) x1 = vec_elem(v, e0 + 2 * k + 1);
+        }
+        __half2 h = __floats2half2_rn(x0, x1);
+        asum += __low2float(h) + __high2float(h);
+        ah[j * AW + k] = *reinterpret_cast<uint32_t*>(&h);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < AW; ++k) af[j * AW + k] = ok ? vec_elem(v, e0 + k) : 0.f;
+    }
+  }
+  const float corr = 1152.f * asum;
+
+  // ---- rows, one ring slot at a time ----
+  const int blk_rows = g.rs * (kRowBlock / g.rs);
+  const int rpg = (g.rs + g.rp - 1) / g.rp;
+  float lm_v = -CUDART_INF_F;
+  int lm_i = 0x7fffffff;
+  for (int r0 = 0; r0 < nrows; r0 += g.rs, ++it) {
+    const int slot = it % kSlots;
+    wait_slot(p, &s.full[slot], (it / kSlots) & 1, (2u << 16) | slot);
+    const int srows = min(g.rs, nrows - r0);
+    const uint8_t* sbuf = s.ring + slot * kSlotBytes;
+    if (active) {
+      const int rb0 = rp * rpg, re = min(rb0 + rpg, srows);
+      for (int r = rb0; r < re; r += 4) {
+        float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        unsigned long long accp[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int j = 0; j < NRMAX; ++j) {
+          const int col = j * g.wpg + wg;
+          if (j < g.nr && col < g.wg_total) {
+            const int boff = (col * 32 + lane) * GB;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              if (r + rr < re) {
+                uint32_t w[GroupWords<GB>::N];
+                lds_group<GB>(sbuf + (size_t)(r + rr) * g.rb + boff, w);
+                if constexpr (I8) dot_i8<GB>(acc[rr][0], acc[rr][1], w, &ah[j * AW]);
+                else dot_bf16<GB>(accp[rr], w, &af[j * AW]);
+              }
+            }
+          }
+        }
+        float a4[4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) a4[rr] = I8 ? (acc[rr][0] + acc[rr][1]) - corr : f2sum(accp[rr]);
+        const float tot = reduce4_rows(a4[0], a4[1], a4[2], a4[3]);
+        const int row = r + ((lane >> 3) & 3);
+        if ((lane & 7) == 0 && row < re) s.part[wg * kRowBlock + ((r0 + row) % blk_rows)] = tot;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[slot]);
+
+    // ---- epilogue of a finished block of rows ----
+    const int done = r0 + srows;
+    if (done % blk_rows == 0 || done == nrows) {
+      bar_compute();
+      const int bs = ((done - 1) / blk_rows) * blk_rows, bn = done - bs;
+      auto rowsum = [&](int rr) {
+        float a = 0.f;
+        for (int w = 0; w < g.wpg; ++w) a += s.part[w * kRowBlock + rr];
+        return I8 && sc ? a * s.scale[bs + rr] : a;
+      };
+      if (op == OP_QKV || op == OP_GU) {
+        for (int pr = tid; pr < bn / 2; pr += kConsumerThreads) {
+          const float v0 = rowsum(2 * pr), v1 = rowsum(2 * pr + 1);
+          const int gr = row0 + bs + 2 * pr;
+          if (op == OP_GU) {
+            const float silu = v0 / (1.f + __expf(-v0));
+            p.act[gr >> 1] = silu * v1;
+          } else {
+            const int hd = p.hd, head = gr / hd, i = (gr % hd) >> 1;
+            if (head < p.Hq + p.Hkv) {
+              const float c = p.rope[((size_t)p.pos * (hd / 2) + i) * 2], sn = p.rope[((size_t)p.pos * (hd / 2) + i) * 2 + 1];
+              const float o0 = v0 * c - v1 * sn, o1 = v1 * c + v0 * sn;
+              if (head < p.Hq) {
+                p.q[head * hd + i] = o0;
+                p.q[head * hd + i + hd / 2] = o1;
+              } else {
+                uint16_t* k = p.kcache + (((size_t)l * p.Hkv + (head - p.Hq)) * p.max_seq + p.pos) * hd;
+                k[i] = f2bf(o0);
+                k[i + hd / 2] = f2bf(o1);
+              }
+            } else {
+              uint16_t* vv = p.vcache + (((size_t)l * p.Hkv + (head - p.Hq - p.Hkv)) * p.max_seq + p.pos) * hd;
+              vv[i] = f2bf(v0);
+              vv[i + hd / 2] = f2bf(v1);
+            }
+          }
+        }
+      } else {
+        for (int rr = tid; rr < bn; rr += kConsumerThreads) {
+          const float val = rowsum(rr);
+          const int gr = row0 + bs + rr;
+          if (op == OP_LM) {
+            if (p.logits) p.logits[gr] = val;
+            if (val > lm_v || (val == lm_v && gr < lm_i)) { lm_v = val; lm_i = gr; }
+          } else {
+            p.x[gr] = __ldcg(p.x + gr) + val;
+          }
+        }
+      }
+      bar_compute();
+    }
+  }
+
+  if (op == OP_LM) {
+    // CTA argmax of this task, folded into the CTA's running best
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, lm_v, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, lm_i, o);
+      if (ov > lm_v || (ov == lm_v && oi < lm_i)) { lm_v = ov; lm_i = oi; }
+    }
+    if (lane == 0) { s.misc->am_v[warp] = lm_v; s.misc->am_i[warp] = lm_i; }
+    bar_compute();
+    if (tid == 0) {
+      float bv = s.misc->lm_v;
+      int bi = s.misc->lm_i;
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float ov = s.misc->am_v[w];
+        const int oi = s.misc->am_i[w];
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      s.misc->lm_v = bv;
+      s.misc->lm_i = bi;
+    }
+    bar_compute();
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Attention (split-KV flash decoding)
+
+__device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : exp2f(m - M); }
+
+// Log-sum-exp merge of the C chunk partials of KV head h into attn_out.
+__device__ void merge_head(const Params& p, int h, int C) {
+  const int G = p.Hq / p.Hkv, hd = p.hd;
+  const int stride = hd + 2;
+  for (int idx = threadIdx.x; idx < G * hd; idx += kConsumerThreads) {
+    const int g = idx / hd, e = idx % hd;
+    float M = -CUDART_INF_F;
+    for (int c = 0; c < C; ++c) {
+      const float* pc = p.attn_part + (((size_t)h * p.kv_chunks_max + c) * G + g) * stride;
+      M = fmaxf(M, __ldcg(pc + hd));
+    }
+    float Ls = 0.f, O = 0.f;
+    for (int c = 0; c < C; ++c) {
+      const float* pc = p.attn_part + (((size_t)h * p.kv_chunks_max + c) * G + g) * stride;
+      const float f = exp2_scale(__ldcg(pc + hd), M);
+      Ls += __ldcg(pc + hd + 1) * f;
+      O += __ldcg(pc + e) * f;
+    }
+    p.attn_out[(h * G + g) * hd + e] = O / Ls;
+  }
+}
+
+template <int HD>
+__device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it) {
+  constexpr int LPP = HD * 2 / 16;       // lanes per position (one 16-byte chunk each)
+  constexpr int PPW = 32 / LPP;          // positions per warp step
+  constexpr int NPS = kSlotBytes / (4 * HD);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cl = lane % LPP, sw = lane / LPP;
+  const int G = p.Hq / p.Hkv;
+  const int h = t.a, c = t.b, l = t.layer;
+  const int P = p.pos + 1;
+  const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
+  if (c >= C) return;
+  int cb, ce;
+  attn_chunk_range(P, C, c, &cb, &ce);
+
+  if (p.sync && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
+
+  // queries of this KV head's group, pre-scaled by log2(e) / sqrt(hd), staged in shared memory
+  // (the GEMV partial-sum region, which attention tasks do not use)
+  const float qs = 1.4426950408889634f * rsqrtf((float)HD);
+  float* qsm = s.part;
+  for (int i = tid; i < G * HD; i += kConsumerThreads) qsm[i] = __ldcg(p.q + h * G * HD + i) * qs;
+  bar_compute();
+
+  float m[kMaxGroup], ls[kMaxGroup], o[kMaxGroup][8];
+#pragma unroll
+  for (int g = 0; g < kMaxGroup; ++g) {
+    m[g] = -CUDART_INF_F;
+    ls[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
+  }
+
+  const size_t head_off = ((size_t)l * p.Hkv + h) * p.max_seq;
+  for (int blk = cb; blk < ce; blk += NPS, ++it) {
+    const int slot = it % kSlots;
+    wait_slot(p, &s.full[slot], (it / kSlots) & 1, (2u << 16) | slot);
+    const int n = min(blk + NPS, ce) - blk;
+    uint8_t* kb = s.ring + slot * kSlotBytes;
+    uint8_t* vb = kb + kSlotBytes / 2;
+    if (p.pos >= blk && p.pos < blk + n) {
+      // this step's own key/value row: written by the QKV stage, read with plain loads
+      const int j = p.pos - blk;
+      if (tid < HD / 4) {
+        const uint2* ks = reinterpret_cast<const uint2*>(p.kcache + (head_off + p.pos) * HD);
+        const uint2* vs = reinterpret_cast<const uint2*>(p.vcache + (head_off + p.pos) * HD);
+        reinterpret_cast<uint2*>(kb + (size_t)j * HD * 2)[tid] = __ldcg(ks + tid);
+        reinterpret_cast<uint2*>(vb + (size_t)j * HD * 2)[tid] = __ldcg(vs + tid);
+        fence_proxy_async_smem();
+      }
+      bar_compute();
+    }
+    for (int base = 0; base < n; base += kConsumerWarps * PPW) {
+      const int j = base + warp * PPW + sw;
+      const bool valid = j < n;
+      float sc[kMaxGroup];
+      {
+        const uint4 kw = valid ? *reinterpret_cast<const uint4*>(kb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
+        const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) {
+          float a = 0.f;
+          if (g < G) {
+            const float4 q0 = *reinterpret_cast<const float4*>(qsm + g * HD + cl * 8);
+            const float4 q1 = *reinterpret_cast<const float4*>(qsm + g * HD + cl * 8 + 4);
+            a = fmaf(q0.x, __uint_as_float(kk[0] << 16), a);
+            a = fmaf(q0.y, __uint_as_float(kk[0] & 0xffff0000u), a);
+            a = fmaf(q0.z, __uint_as_float(kk[1] << 16), a);
+            a = fmaf(q0.w, __uint_as_float(kk[1] & 0xffff0000u), a);
+            a = fmaf(q1.x, __uint_as_float(kk[2] << 16), a);
+            a = fmaf(q1.y, __uint_as_float(kk[2] & 0xffff0000u), a);
+            a = fmaf(q1.z, __uint_as_float(kk[3] << 16), a);
+            a = fmaf(q1.w, __uint_as_float(kk[3] & 0xffff0000u), a);
+          }
+#pragma unroll
+          for (int off = 1; off < LPP; off <<= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+          sc[g] = a;
+        }
+      }
+      if (valid) {
+        const uint4 vw = *reinterpret_cast<const uint4*>(vb + (size_t)j * HD * 2 + cl * 16);
+        const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) {
+          if (g < G) {
+            const float mn = fmaxf(m[g], sc[g]);
+            const float cr = exp2_scale(m[g], mn), pe = exp2f(sc[g] - mn);
+            ls[g] = ls[g] * cr + pe;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              o[g][2 * q] = fmaf(o[g][2 * q], cr, pe * __uint_as_float(vv[q] << 16));
+              o[g][2 * q + 1] = fmaf(o[g][2 * q + 1], cr, pe * __uint_as_float(vv[q] & 0xffff0000u));
+            }
+            m[g] = mn;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[slot]);
+  }
+
+  // merge the sub-warps of this warp (lanes with the same chunk)
+#pragma unroll
+  for (int g = 0; g < kMaxGroup; ++g) {
+#pragma unroll
+    for (int off = LPP; off < 32; off <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, ls[g], off);
+      const float M = fmaxf(m[g], mo);
+      const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
+      ls[g] = ls[g] * fa + lo * fb;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float oo = __shfl_xor_sync(0xffffffffu, o[g][e], off);
+        o[g][e] = o[g][e] * fa + oo * fb;
+      }
+      m[g] = M;
+    }
+  }
+  // merge the 16 warps: a 4-round tree through shared memory
+  const int stride = HD + 2;
+  for (int k = kConsumerWarps / 2; k >= 1; k >>= 1) {
+    if (warp >= k && warp < 2 * k && sw == 0) {
+      float* ent = s.aux + (size_t)(warp - k) * kMaxGroup * stride;
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) {
+        if (g < G) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
+          if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
+        }
+      }
+    }
+    bar_compute();
+    if (warp < k) {
+      const float* ent = s.aux + (size_t)warp * kMaxGroup * stride;
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) {
+        if (g < G) {
+          const float mo = ent[g * stride + HD], lo = ent[g * stride + HD + 1];
+          const float M = fmaxf(m[g], mo);
+          const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
+          ls[g] = ls[g] * fa + lo * fb;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[g][e] = o[g][e] * fa + ent[g * stride + cl * 8 + e] * fb;
+          m[g] = M;
+        }
+      }
+    }
+    bar_compute();
+  }
+  // this CTA's partial
+  if (warp == 0 && sw == 0) {
+    float* dst = p.attn_part + ((size_t)h * p.kv_chunks_max + c) * G * stride;
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+      if (g < G) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[g * stride + cl * 8 + e] = o[g][e];
+        if (cl == 0) { dst[g * stride + HD] = m[g]; dst[g * stride + HD + 1] = ls[g]; }
+      }
+    }
+  }
+  if (!p.sync) return;
+  // ticket: the last chunk of this head to finish merges all of them and signals
+  bar_compute();
+  uint32_t* ticket = p.attn_ticket + l * p.Hkv + h;
+  if (tid == 0) {
+    __threadfence();
+    const uint32_t old = atomicAdd(ticket, 1u);
+    s.misc->flag = (old == (uint32_t)(C - 1));
+  }
+  bar_compute();
+  if (s.misc->flag) {
+    __threadfence();
+    merge_head(p, h, C);
+    bar_compute();
+    if (tid == 0) {
+      *ticket = 0u;
+      __threadfence();
+      atomicAdd(p.ctr + t.sig_ctr, 1u);
+    }
+  }
+  bar_compute();
+}
+
+// ------------------------------------------------------------------------------------------------
+// Grid argmax of the per-CTA LM maxima (lowest index on ties)
+
+__device__ void grid_argmax(const Params& p, Smem& s) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  float bv = -CUDART_INF_F;
+  int bi = 0x7fffffff;
+  for (int b = lane; b < p.grid; b += 32) {
+    const float v = __ldcg(p.am_val + b);
+    const int i = __ldcg(p.am_idx + b);
+    if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  if (lane == 0) *p.next_token = (bi >= 0 && bi < p.V) ? bi : -1;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Compute warps
+
+__device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    int tok = p.token;
+    if (tok < 0) tok = __ldcg(p.next_token);
+    if (tok < 0 || tok >= p.V) {
+      raise_abort(p, (4u << 16));
+      tok = 0;
+    }
+    s.misc->token = tok;
+    s.misc->lm_v = -CUDART_INF_F;
+    s.misc->lm_i = 0x7fffffff;
+  }
+  bar_compute();
+  const int token = s.misc->token;
+  if (p.init_x) {
+    const int r0 = p.o_rows[2 * blockIdx.x], n = p.o_rows[2 * blockIdx.x + 1];
+    for (int r = tid; r < n; r += kConsumerThreads) p.x[r0 + r] = bf2f(p.embed[(size_t)token * p.d + r0 + r]);
+  }
+  uint32_t it = 0;
+  const bool i8 = p.wdtype == AMK_W_INT8;
+  for (int ti = 0; ti < nt; ++ti) {
+    const Task t = tasks[ti];
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_tasks_per_cta + ti) * 4 : nullptr;
+    if (tr && tid == 0) { tr[0] = ((unsigned long long)t.op << 32) | (unsigned long long)t.layer << 16 | (unsigned)ti; tr[1] = globaltimer(); }
+    if (is_gemv(t.op)) {
+      const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
+      const bool w8 = i8 && !(t.op == OP_LM && p.tied);
+      if (w8) {
+        switch (g.gb) {
+          case 16: gemv_task<true, 16>(p, t, s, it, token); break;
+          case 8: gemv_task<true, 8>(p, t, s, it, token); break;
+          case 4: gemv_task<true, 4>(p, t, s, it, token); break;
+          default: gemv_task<true, 2>(p, t, s, it, token); break;
+        }
+      } else {
+        switch (g.gb) {
+          case 16: gemv_task<false, 16>(p, t, s, it, token); break;
+          case 8: gemv_task<false, 8>(p, t, s, it, token); break;
+          default: gemv_task<false, 4>(p, t, s, it, token); break;
+        }
+      }
+      if (tr && tid == 0) tr[2] = globaltimer();
+      if (t.op == OP_LM) {
+        if (t.flags & kLastOfStage) {
+          if (tid == 0) { p.am_val[blockIdx.x] = s.misc->lm_v; p.am_idx[blockIdx.x] = s.misc->lm_i; }
+          if (p.sync) {
+            bar_compute();
+            if (tid == 0) {
+              __threadfence();
+              const uint32_t old = atomicAdd(p.am_ticket, 1u);
+              s.misc->flag = (old == (uint32_t)(p.grid - 1));
+            }
+            bar_compute();
+            if (s.misc->flag) {
+              __threadfence();
+              grid_argmax(p, s);
+              if (tid == 0) *p.am_ticket = 0u;
+            }
+          }
+        }
+      } else if (p.sync && (t.flags & kLastOfStage) && t.sig_ctr >= 0) {
+        bar_compute();
+        signal_counter(p, t.sig_ctr);
+      }
+    } else if (t.op == OP_ATTN) {
+      if (p.hd == 64) attn_task<64>(p, t, s, it);
+      else attn_task<128>(p, t, s, it);
+      if (tr && tid == 0) tr[2] = globaltimer();
+    } else if (t.op == OP_MERGE) {
+      merge_head(p, t.a, attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max));
+    } else if (t.op == OP_ARGMAX) {
+      grid_argmax(p, s);
+    }
+    if (tr && tid == 0) tr[3] = globaltimer();
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Smem s = carve(smem_raw);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], kConsumerWarps);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+  const int b = blockIdx.x;
+  const Task* tasks = p.tasks + p.task_off[b];
+  const int nt = p.task_off[b + 1] - p.task_off[b];
+  if (threadIdx.x >= kConsumerThreads) {
+    if (threadIdx.x == kConsumerThreads) producer(p, tasks, nt, s);
+    return;
+  }
+  compute(p, tasks, nt, s);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Weight packer: one CTA per packed row.
+
+__global__ void pack_kernel(int role, int hd, int ffn, const void* src, int src_dtype, int cols, int dst_dtype,
+                            void* dst, uint16_t* scales) {
+  __shared__ float red[32];
+  const int pr = blockIdx.x;
+  const int sr = packed_row_source(role, hd, ffn, pr);
+  auto load = [&](int k) -> float {
+    if (src_dtype == AMK_SRC_F32) return static_cast<const float*>(src)[(size_t)sr * cols + k];
+    return bf2f(static_cast<const uint16_t*>(src)[(size_t)sr * cols + k]);
+  };
+  if (dst_dtype == AMK_W_BF16) {
+    uint16_t* out = static_cast<uint16_t*>(dst) + (size_t)pr * cols;
+    for (int k = threadIdx.x; k < cols; k += blockDim.x) out[k] = f2bf(load(k));
+    return;
+  }
+  float amax = 0.f;
+  for (int k = threadIdx.x; k < cols; k += blockDim.x) amax = fmaxf(amax, fabsf(load(k)));
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (threadIdx.x == 0) red[0] = a;
+  }
+  __syncthreads();
+  const uint16_t sb = f2bf(__fdiv_rn(red[0], 127.f));
+  const float s = bf2f(sb);
+  if (threadIdx.x == 0) scales[pr] = sb;
+  int8_t* out = static_cast<int8_t*>(dst) + (size_t)pr * cols;
+  for (int k = threadIdx.x; k < cols; k += blockDim.x) {
+    float q = 0.f;
+    if (s > 0.f) q = fminf(127.f, fmaxf(-127.f, rintf(__fdiv_rn(load(k), s))));
+    out[k] = (int8_t)q;
+  }
+}
+
+}  // namespace dev
+
+// ------------------------------------------------------------------------------------------------
+// Host-side launch helpers (called from amk_api.cu)
+
+cudaError_t prepare_kernel_attributes() {
+  return cudaFuncSetAttribute(dev::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+cudaError_t occupancy(int* blocks_per_sm) {
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, dev::decode_kernel, kThreads, kSmemBytes);
+}
+
+cudaError_t launch_decode(const Params& p, cudaStream_t stream, bool cooperative) {
+  void* args[] = {const_cast<Params*>(&p)};
+  if (cooperative)
+    return cudaLaunchCooperativeKernel((const void*)dev::decode_kernel, dim3(p.grid), dim3(kThreads), args, kSmemBytes,
+                                       stream);
+  return cudaLaunchKernel((const void*)dev::decode_kernel, dim3(p.grid), dim3(kThreads), args, kSmemBytes, stream);
+}
+
+cudaError_t launch_pack(int role, int hd, int ffn, const void* src, int src_dtype, int rows, int cols, int dst_dtype,
+                        void* dst, void* scales, cudaStream_t stream) {
+  dev::pack_kernel<<<rows, 256, 0, stream>>>(role, hd, ffn, src, src_dtype, cols, dst_dtype, dst,
+                                             static_cast<uint16_t*>(scales));
+  return cudaGetLastError();
+}
+
+}  // namespace amk

@@ -1,0 +1,181 @@
+// Internal layout shared by the host planner, the host API and the device code of libamk.
+//
+// The persistent kernel follows the Layer-0 design of "AutoMegaKernel: A Statically-Checked Agent
+// Harness for Self-Retargeting Megakernel Synthesis" (technical summary, "Methodology"): one CTA per
+// SM walks its own task list in a globally valid order, each task doing wait -> dispatch -> signal
+// on monotonic counters. Here the task list is a fixed per-layer pattern built on the host:
+//   per layer l:  QKV(l) -> ATTN(l) -> O(l) -> GU(l) -> DOWN(l);   then LM (head + argmax).
+// Every GEMV stage is row-split over all CTAs; ATTN is split over (KV head, KV chunk).
+#pragma once
+#include <stdint.h>
+
+#include "../../include/amk.h"
+
+#ifdef __CUDACC__
+#define AMK_HD __host__ __device__
+#else
+#define AMK_HD
+#endif
+
+namespace amk {
+
+// ---- CTA shape and shared-memory budget ------------------------------------------------------
+constexpr int kConsumerWarps   = 16;
+constexpr int kConsumerThreads = kConsumerWarps * 32;      // 512 compute threads
+constexpr int kThreads         = kConsumerThreads + 32;    // + 1 producer (bulk-copy) warp
+constexpr int kSlotBytes       = 32768;                    // one bulk-copy ring slot
+constexpr int kSlots           = 6;                        // ring depth (192 KB in flight per SM)
+constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block
+constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV task (scale cache)
+constexpr int kMaxGroup        = 4;                        // Hq / Hkv supported
+constexpr int kAuxBytes        = 8 * kMaxGroup * (128 + 2) * 4;   // attention cross-warp tree
+constexpr int kRingBytes       = kSlots * kSlotBytes;
+constexpr int kPartBytes       = kConsumerWarps * kRowBlock * 4;
+constexpr int kScaleBytes      = kMaxTaskRows * 4;
+constexpr int kMiscBytes       = 512;
+constexpr int kSmemBytes       = kRingBytes + kPartBytes + kAuxBytes + kScaleBytes + kMiscBytes;
+
+// ---- tasks -----------------------------------------------------------------------------------
+enum Op : uint16_t {
+  OP_QKV = 1,     // RMSNorm(x)*g1 -> packed QKV GEMV -> RoPE -> q scratch, K/V cache at pos
+  OP_ATTN = 2,    // GQA attention of one KV head over one KV chunk -> partial (m, l, o)
+  OP_O = 3,       // O GEMV + residual into x
+  OP_GU = 4,      // RMSNorm(x)*g2 -> gate/up GEMV -> SwiGLU -> act scratch
+  OP_DOWN = 5,    // down GEMV + residual into x
+  OP_LM = 6,      // RMSNorm(x)*gf -> LM-head GEMV -> logits + per-CTA argmax
+  OP_MERGE = 7,   // (op-per-kernel ablation only) log-sum-exp merge of one KV head's partials
+  OP_ARGMAX = 8,  // (op-per-kernel ablation only) grid argmax of the per-CTA maxima
+};
+
+// GEMV op index into Params::geom
+AMK_HD inline int gemv_slot_of(int op) {
+  return op == OP_QKV ? 0 : op == OP_O ? 1 : op == OP_GU ? 2 : op == OP_DOWN ? 3 : 4;
+}
+
+// Counters: per layer one per stage kind, then nothing else (the argmax and the attention merge
+// use tickets, which the last arriver resets).
+enum CtrKind { CTR_QKV = 0, CTR_ATTN = 1, CTR_O = 2, CTR_GU = 3, CTR_DOWN = 4, CTR_PER_LAYER = 5 };
+
+struct Task {
+  uint16_t op;
+  uint16_t layer;
+  int32_t  a;          // GEMV: first packed row;  ATTN: KV head;  MERGE: KV head
+  int32_t  b;          // GEMV: number of rows;    ATTN: chunk index
+  int32_t  wait_ctr;   // counter to wait on, -1 = none
+  uint32_t wait_mult;  // wait until counter >= epoch * wait_mult (mod 2^32)
+  int32_t  sig_ctr;    // counter to add 1 to when done, -1 = none
+  uint32_t flags;      // kFirstOfStage | kLastOfStage: only the first task of a stage on a CTA
+                       // waits, only the last signals (a stage split into several tasks on one
+                       // CTA still signals once)
+  uint32_t pad;
+};
+constexpr uint32_t kFirstOfStage = 1u;
+constexpr uint32_t kLastOfStage = 2u;
+
+// How one GEMV shape maps onto the 512 compute threads. A row of `rb` bytes is cut into groups of
+// `gb` bytes (one shared-memory vector load per thread); `wg_total` warps' worth of groups cover a
+// row. Warps form `rp` row groups of `wpg` warps; a thread keeps the activations of its groups in
+// registers for the whole task (`nr` groups per thread).
+struct GemvGeom {
+  int32_t K;         // elements per row
+  int32_t rb;        // bytes per row
+  int32_t gb;        // bytes per group: 16, 8, 4 or 2
+  int32_t wg_total;  // (rb / gb) / 32
+  int32_t wpg;       // warps per row group
+  int32_t nr;        // groups per thread
+  int32_t rp;        // row groups
+  int32_t rs;        // rows per ring slot
+};
+
+struct LayerPtrs {
+  const void*     wqkv;
+  const void*     wo;
+  const void*     wgu;
+  const void*     wdown;
+  const uint16_t* sqkv;
+  const uint16_t* so;
+  const uint16_t* sgu;
+  const uint16_t* sdown;
+  const uint16_t* attn_norm;
+  const uint16_t* ffn_norm;
+};
+
+struct Params {
+  // model
+  int L, d, Hq, Hkv, hd, ffn, V, max_seq;
+  float eps;
+  int wdtype;          // AMK_W_INT8 / AMK_W_BF16
+  int tied;
+  int grid;
+  const LayerPtrs* layers;     // device [L]
+  const uint16_t* embed;       // bf16 [V, d]
+  const uint16_t* final_norm;  // bf16 [d]
+  const void*     lm_w;        // packed head or the embedding when tied
+  const uint16_t* lm_s;        // scales or null
+  uint16_t* kcache;            // bf16 [L][Hkv][max_seq][hd]
+  uint16_t* vcache;
+  const float* rope;           // interleaved (cos, sin) [max_seq][hd/2][2]
+  // scratch (device)
+  float* x;                    // residual stream [d]
+  float* q;                    // roped queries [Hq*hd]
+  float* attn_out;             // merged attention [Hq*hd]
+  float* act;                  // SwiGLU output [ffn]
+  float* attn_part;            // [Hkv][kv_chunks_max][G][hd + 2]
+  float* am_val;               // per-CTA LM maxima [grid]
+  int*   am_idx;
+  uint32_t* ctr;               // [L * CTR_PER_LAYER]
+  uint32_t* attn_ticket;       // [L * Hkv]
+  uint32_t* am_ticket;         // [1]
+  uint32_t* abort_flag;        // device word: nonzero after a wait expired
+  volatile uint32_t* status;   // host-mapped sticky status word
+  unsigned long long* trace;   // [grid][max_tasks_per_cta][4] or null
+  int max_tasks_per_cta;
+  // plan
+  const Task* tasks;           // this launch's task list
+  const int*  task_off;        // [grid + 1]
+  GemvGeom geom[5];            // QKV, O, GU, DOWN, LM
+  int kv_block;
+  int kv_chunks_max;
+  unsigned long long timeout_ns;
+  // per launch
+  uint32_t epoch;
+  int token;                   // >= 0, or -1 to read *next_token
+  int pos;
+  float* logits;               // may be null
+  int*   next_token;
+  int sync;                    // 1 = persistent megakernel (waits/signals), 0 = op-per-kernel
+  int init_x;                  // this launch writes x = E[token] for its O rows first
+  const int* o_rows;           // [grid][2] (row0, nrows) of each CTA's O tasks (for init_x)
+};
+
+// ---- shared host/device helpers ----------------------------------------------------------------
+AMK_HD inline int packed_row_source(int role, int hd, int ffn, int packed_row) {
+  if (role == AMK_ROLE_QKV) {
+    int head = packed_row / hd, j = packed_row % hd;
+    return head * hd + ((j & 1) ? (j >> 1) + hd / 2 : (j >> 1));
+  }
+  if (role == AMK_ROLE_GATE_UP) return (packed_row & 1) ? ffn + (packed_row >> 1) : (packed_row >> 1);
+  return packed_row;
+}
+
+// Attention chunking of positions 0..P-1 of one KV head: chunks of cs = ceil(P / c) positions,
+// c = min(cmax, ceil(P / kv_block)); the count returned is ceil(P / cs), so no chunk is empty.
+AMK_HD inline int attn_num_chunks(int P, int kv_block, int cmax) {
+  if (P < 1) return 1;
+  int c = (P + kv_block - 1) / kv_block;
+  if (c > cmax) c = cmax;
+  if (c < 1) c = 1;
+  int cs = (P + c - 1) / c;
+  return (P + cs - 1) / cs;
+}
+AMK_HD inline void attn_chunk_range(int P, int C, int c, int* begin, int* end) {
+  int cs = (P + C - 1) / C;
+  int b = c * cs, e = b + cs;
+  if (b > P) b = P;
+  if (e > P) e = P;
+  *begin = b;
+  *end = e;
+}
+AMK_HD inline int attn_positions_per_slot(int hd) { return kSlotBytes / (2 * hd * 2); }
+
+}  // namespace amk

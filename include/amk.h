@@ -1,0 +1,208 @@
+/*
+ * amk.h — C ABI of libamk: batch-1 Llama-family decode as ONE persistent CUDA launch (sm_100a).
+ *
+ * Source of the operation. "AutoMegaKernel: A Statically-Checked Agent Harness for Self-Retargeting
+ * Megakernel Synthesis" (abstract) compiles the whole forward pass of a HuggingFace Llama-family model
+ * into a single persistent cooperative kernel for greedy decode, with an int8 weight-only (W8A16)
+ * variant; its technical summary ("Problem Statement") fixes the workload as single-stream
+ * autoregressive decoding at batch size 1, whose floor is weight bytes / HBM bandwidth, and its
+ * "Methodology" (Layer 0) describes one block per SM walking a task order with wait -> dispatch ->
+ * signal on monotonic counters. The pages print no API; the calls below are this library's own.
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA device addresses on the current device; host pointers are ordinary
+ *     host memory. `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - The caller owns every buffer it passes (weights, KV cache, logits, token). A handle owns only
+ *     what amk_create allocates (task list, counters, scratch, RoPE table, status word) and
+ *     amk_destroy frees exactly that.
+ *   - Return codes: AMK_OK (0) or a negative AMK_ERR_*. Argument errors are detected on the host
+ *     before anything is launched. Launches are asynchronous: a device-side failure (a bounded wait
+ *     that ran out) is sticky and is reported by the next amk_decode_step* call and by amk_status.
+ *   - Not thread-safe per handle: one handle must not be used from two host threads at once.
+ */
+#ifndef AMK_H_
+#define AMK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ---------------------------------------------------------------------------- */
+#define AMK_OK                   0
+#define AMK_ERR_INVALID_ARG     -1  /* bad pointer, size, alignment, token or position */
+#define AMK_ERR_CUDA            -2  /* a CUDA runtime call failed (see amk_last_cuda_error) */
+#define AMK_ERR_NOT_RESIDENT    -3  /* the persistent grid cannot be co-resident (1 CTA per SM) */
+#define AMK_ERR_DEVICE_TIMEOUT  -4  /* a bounded device wait expired; the handle is unusable */
+#define AMK_ERR_UNSUPPORTED     -5  /* dims outside what the kernels support (see amk_create) */
+#define AMK_ERR_PLAN            -6  /* the static task-list check rejected the plan */
+#define AMK_ERR_NO_MEMORY       -7  /* host or device allocation failed */
+
+/* ---- enums ----------------------------------------------------------------------------------- */
+#define AMK_W_INT8   0   /* int8 weights, one bf16 scale per output row (W8A16) */
+#define AMK_W_BF16   1   /* bf16 weights, no scales */
+
+#define AMK_SRC_F32  0   /* packer source element type: fp32 */
+#define AMK_SRC_BF16 1   /* packer source element type: bf16 */
+
+/* Weight roles: each selects the packed row order the kernels expect (see amk_pack_weight). */
+#define AMK_ROLE_PLAIN    0  /* row-major, rows in source order                                   */
+#define AMK_ROLE_QKV      1  /* source = [Wq; Wk; Wv] rows; per head, rows i and i+hd/2 adjacent   */
+#define AMK_ROLE_O        2  /* source = Wo [d, Hq*hd], source order                               */
+#define AMK_ROLE_GATE_UP  3  /* source = [Wgate; Wup] rows; gate row i and up row i adjacent       */
+#define AMK_ROLE_DOWN     4  /* source = Wdown [d, ffn], source order                              */
+#define AMK_ROLE_LM_HEAD  5  /* source = lm_head [V, d], source order                              */
+
+/* ---- model description ----------------------------------------------------------------------- */
+typedef struct amk_dims {
+  int   n_layers;      /* L >= 1                                                              */
+  int   d_model;       /* d, a multiple of 64                                                 */
+  int   n_q_heads;     /* Hq, a multiple of n_kv_heads                                        */
+  int   n_kv_heads;    /* Hkv >= 1; Hq / Hkv in 1..4                                          */
+  int   head_dim;      /* hd in {64, 128}                                                     */
+  int   ffn;           /* SwiGLU hidden size, a multiple of 64                                */
+  int   vocab;         /* V >= 1                                                              */
+  int   max_seq;       /* KV cache capacity in positions (>= 1)                               */
+  float rope_theta;    /* RoPE base (rotate-half form, no scaling)                            */
+  float rms_eps;       /* RMSNorm epsilon                                                     */
+  int   weight_dtype;  /* AMK_W_INT8 or AMK_W_BF16 for every linear weight                   */
+  int   tied_head;     /* 1: the LM head is the bf16 embedding table; 0: lm_head is given     */
+} amk_dims;
+
+/* Device pointers of one model. Per-layer entries are HOST arrays of n_layers DEVICE pointers;
+ * amk_create copies the pointer values, so the arrays may be freed after it returns.
+ * Packed weights and scales come from amk_pack_weight with the matching role. All device
+ * pointers must be 16-byte aligned. */
+typedef struct amk_weights {
+  const void*        embed;       /* bf16 [V, d]                                            */
+  const void* const* attn_norm;   /* [L] bf16 [d]                                           */
+  const void* const* ffn_norm;    /* [L] bf16 [d]                                           */
+  const void*        final_norm;  /* bf16 [d]                                               */
+  const void* const* wqkv;        /* [L] packed AMK_ROLE_QKV,     [(Hq+2Hkv)*hd, d]          */
+  const void* const* wo;          /* [L] packed AMK_ROLE_O,       [d, Hq*hd]                 */
+  const void* const* wgu;         /* [L] packed AMK_ROLE_GATE_UP, [2*ffn, d]                 */
+  const void* const* wdown;       /* [L] packed AMK_ROLE_DOWN,    [d, ffn]                   */
+  const void*        lm_head;     /* packed AMK_ROLE_LM_HEAD [V, d]; NULL when tied_head    */
+  const void* const* sqkv;        /* [L] bf16 scales in packed row order; NULL for bf16     */
+  const void* const* so;
+  const void* const* sgu;
+  const void* const* sdown;
+  const void*        slm;         /* bf16 [V]; NULL when tied_head or bf16                   */
+  void*              k_cache;     /* bf16 [L][Hkv][max_seq][hd], read and written            */
+  void*              v_cache;     /* bf16 [L][Hkv][max_seq][hd], read and written            */
+} amk_weights;
+
+/* Optional tuning and test knobs; pass NULL to amk_create for the defaults (all fields 0). */
+typedef struct amk_options {
+  int grid;              /* persistent CTAs; 0 = one per SM                                    */
+  int kv_block;          /* minimum positions per attention chunk; 0 = 64                      */
+  int max_kv_chunks;     /* cap on attention chunks per KV head; 0 = grid / Hkv                */
+  int timeout_ms;        /* bound on every device wait; 0 = 2000 ms                            */
+  int trace;             /* 1: record per-task timestamps (see amk_trace_read)                 */
+  int test_drop_signal;  /* TEST ONLY: 1 + index of a counter signal the planner omits, so the
+                            waits on it expire with AMK_ERR_DEVICE_TIMEOUT; 0 = off            */
+} amk_options;
+
+typedef struct amk_handle amk_handle;
+
+/* ---- packing --------------------------------------------------------------------------------- */
+
+/* Bytes of the packed weight buffer for `rows` x `cols` in `dst_dtype` (rows * cols * 1 or 2). */
+size_t amk_packed_bytes(int rows, int cols, int dst_dtype);
+
+/* Source row that lands in packed row `packed_row` for `role` (host-only helper, no GPU).
+ * Returns -1 on bad arguments. For AMK_ROLE_QKV, within each head of hd rows, packed rows
+ * 2i and 2i+1 hold source rows i and i + hd/2; for AMK_ROLE_GATE_UP packed rows 2i and 2i+1
+ * hold gate row i (source row i) and up row i (source row ffn + i). */
+int amk_packed_row_source(int role, const amk_dims* dims, int rows, int packed_row);
+
+/* Device-side weight packer (W8A16 quantiser / bf16 copier).
+ *   src:        device, [rows, cols] row-major in `src_dtype`; for QKV the rows of Wq, Wk, Wv
+ *               stacked, for GATE_UP the rows of Wgate then Wup.
+ *   packed_out: device, amk_packed_bytes(rows, cols, dst_dtype) bytes, rows in the role's order.
+ *   scales_out: device bf16 [rows] (packed order) for AMK_W_INT8; ignored (may be NULL) for bf16.
+ * int8: s = bf16_rne(max|w_row| / 127), q = clamp(rint(w / s), -127, 127); s = 0, q = 0 for a row
+ * whose scale rounds to 0. bf16: round-to-nearest-even of each element.
+ * `dims` may be NULL for AMK_ROLE_PLAIN; for other roles rows/cols must match dims.
+ * Asynchronous on `stream`. */
+int amk_pack_weight(int role, const amk_dims* dims, const void* src, int src_dtype, int rows, int cols,
+                    int dst_dtype, void* packed_out, void* scales_out, void* stream);
+
+/* ---- handle lifetime ------------------------------------------------------------------------- */
+
+/* Validates dims/pointers, builds and statically checks the per-CTA task list, allocates the
+ * handle's device state and checks that the persistent grid is co-resident. Synchronous.
+ * Supported: head_dim in {64,128}; Hq/Hkv in 1..4; d_model, ffn and Hq*hd multiples of 64 and
+ * at most 16384; weight rows of at most 32 KB. On failure *out is NULL. */
+int  amk_create(const amk_dims* dims, const amk_weights* weights, const amk_options* options,
+                amk_handle** out);
+
+/* Frees the handle's own device and host state (never the caller's buffers). Synchronizes the
+ * device first. NULL is ignored. */
+void amk_destroy(amk_handle* h);
+
+/* ---- the decode step ------------------------------------------------------------------------- */
+
+/* One greedy decode step in ONE persistent launch on `stream`.
+ *   token_id:       token at position `pos`, in [0, V); or -1 to read it from *next_token_out
+ *                   (written by the previous step on the same stream: device-side feedback).
+ *   pos:            absolute position, 0 <= pos < max_seq. K/V are written at `pos` and attention
+ *                   covers positions 0..pos (positions < pos must hold earlier keys/values).
+ *   logits_out:     device fp32 [V], or NULL to skip writing logits.
+ *   next_token_out: device int32 [1], receives argmax(logits) (lowest index on ties). Required.
+ * Returns AMK_ERR_DEVICE_TIMEOUT if an earlier launch of this handle expired a wait. */
+int  amk_decode_step(amk_handle* h, int token_id, int pos, float* logits_out, int* next_token_out,
+                     void* stream);
+
+/* Ablation: the same step with the same device routines, launched one kernel per operation
+ * (per layer: QKV, attention partials, attention merge, O, gate/up, down; then LM head and the
+ * argmax), so activations cross HBM between kernels and there is no cross-SM counter. */
+int  amk_decode_step_unfused(amk_handle* h, int token_id, int pos, float* logits_out,
+                             int* next_token_out, void* stream);
+
+/* Sticky device status without synchronizing: AMK_OK or AMK_ERR_DEVICE_TIMEOUT (a wait expired in
+ * an earlier launch). `detail` (may be NULL) receives the raw status word: bits 0..15 the counter
+ * or slot index that expired, bits 16..23 the wait kind (1 counter, 2 full slot, 3 empty slot). */
+int  amk_status(const amk_handle* h, uint32_t* detail);
+
+/* Last CUDA error string seen by this library on this thread ("" if none). */
+const char* amk_last_cuda_error(void);
+
+/* ---- plan introspection (host-only) ---------------------------------------------------------- */
+
+typedef struct amk_plan_info {
+  int      grid;              /* persistent CTAs                                          */
+  int      threads;           /* threads per CTA                                          */
+  int      smem_bytes;        /* dynamic shared memory per CTA                            */
+  int      n_tasks;           /* tasks over all CTAs                                      */
+  int      n_counters;        /* inter-CTA counters                                       */
+  int      kv_chunks_max;     /* attention chunks per KV head at most                     */
+  uint64_t weight_bytes;      /* weight + scale + embedding-row + gain bytes one step reads */
+} amk_plan_info;
+
+int amk_plan_info_get(const amk_handle* h, amk_plan_info* out);
+
+/* Bytes one decode step at `pos` must read: weights (+scales), one embedding row, the norm
+ * gains and the KV cache over positions 0..pos of every layer. Host-only, no GPU. */
+uint64_t amk_step_bytes(const amk_dims* dims, int pos);
+
+/* Static task-list check without a GPU: builds the plan for `dims` on `grid` CTAs, optionally
+ * plants one defect (mutation 0 = none; 1 drop a signal, 2 raise a wait threshold above its
+ * producer count, 3 swap two tasks of one CTA against stage order, 4 make a wait refer to a
+ * later stage, 5 drop a stage's producer), runs the checker and writes its verdict to `msg`.
+ * Returns AMK_OK when the plan is accepted, AMK_ERR_PLAN when it is rejected. */
+int amk_plan_check(const amk_dims* dims, int grid, int mutation, char* msg, int msg_len);
+
+/* ---- tracing --------------------------------------------------------------------------------- */
+
+/* With options.trace = 1, every CTA records (task, wait-start, wait-end, done) %globaltimer
+ * stamps of the last step. Copies up to `max_records` records of 4 uint64 each into the host
+ * buffer `out` (synchronizes the device) and returns how many were written, or a negative code. */
+int amk_trace_read(amk_handle* h, uint64_t* out, int max_records);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AMK_H_ */

@@ -251,12 +251,13 @@ def decode_step(model: OracleModel, kv: OracleKV, token: int, pos: int) -> torch
 
 
 def full_forward(model: OracleModel, tokens: List[int], start: int = 0, prefix: Optional[OracleKV] = None,
-                 store=bf16_round) -> torch.Tensor:
+                 store=bf16_round, kv_out: Optional[OracleKV] = None) -> torch.Tensor:
     """Logits [T, V] of a causal forward over `tokens` at positions start..start+T-1, all at once.
 
     A second, independent formulation: every position's q/k/v in one matmul per layer, then a masked
     [T, start+T] softmax per head. Keys/values of the new positions pass through `store` exactly as
-    the step-wise cache does; positions < start come from `prefix`.
+    the step-wise cache does; positions < start come from `prefix`. If `kv_out` is given, the stored
+    keys/values of positions 0..start+T-1 are written into it (a prompt's cache in one pass).
     """
     cfg = model.cfg
     hq, hkv, hd = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
@@ -279,6 +280,9 @@ def full_forward(model: OracleModel, tokens: List[int], start: int = 0, prefix: 
             vv[:, :start] = prefix.v[l][:, :start]
         kk[:, start:] = store(k).permute(1, 0, 2)
         vv[:, start:] = store(v).permute(1, 0, 2)
+        if kv_out is not None:
+            kv_out.k[l][:, :P] = kk
+            kv_out.v[l][:, :P] = vv
         mask = torch.arange(P)[None, :] <= torch.tensor(positions)[:, None]   # [T, P]
         o = torch.empty(T, hq, hd, dtype=F32)
         for i in range(hq):

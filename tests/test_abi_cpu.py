@@ -1,0 +1,104 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared call, and its host-only
+logic (packed row order, byte model, argument checks, the static task-list checker) behaves."""
+import ctypes as C
+
+import pytest
+
+from decode_megakernel_launch_b200 import synth
+
+amk = pytest.importorskip("decode_megakernel_launch_b200.amk", reason="libamk.so not built")
+from decode_megakernel_launch_b200.runtime import dims_of  # noqa: E402
+
+CONFIGS = ["tiny", "smollm135m", "llama1b", "llama8b", "llama1b_long32k"]
+
+
+def test_every_declared_symbol_is_exported():
+    names = amk.exported_symbols_in_header()
+    assert "amk_decode_step" in names and "amk_create" in names
+    for n in names:
+        assert hasattr(amk.lib, n), n
+
+
+def test_packed_bytes():
+    assert amk.amk_packed_bytes(6144, 4096, amk.AMK_W_INT8) == 6144 * 4096
+    assert amk.amk_packed_bytes(6144, 4096, amk.AMK_W_BF16) == 2 * 6144 * 4096
+    assert amk.amk_packed_bytes(-1, 4, amk.AMK_W_INT8) == 0
+    assert amk.amk_packed_bytes(4, 4, 7) == 0
+
+
+def test_packed_row_order_is_a_pairing_permutation():
+    cfg = synth.preset("llama8b")
+    d = dims_of(cfg)
+    rows = cfg.qkv_rows
+    src = [amk.amk_packed_row_source(amk.AMK_ROLE_QKV, C.byref(d), rows, r) for r in range(rows)]
+    assert sorted(src) == list(range(rows))
+    hd = cfg.head_dim
+    for r in range(0, rows, 2):
+        head = r // hd
+        i = (r % hd) // 2
+        assert src[r] == head * hd + i and src[r + 1] == head * hd + i + hd // 2
+    gu = [amk.amk_packed_row_source(amk.AMK_ROLE_GATE_UP, C.byref(d), 2 * cfg.ffn, r) for r in range(2 * cfg.ffn)]
+    assert gu[:4] == [0, cfg.ffn, 1, cfg.ffn + 1] and sorted(gu) == list(range(2 * cfg.ffn))
+    assert amk.amk_packed_row_source(amk.AMK_ROLE_O, C.byref(d), 10, 7) == 7
+    assert amk.amk_packed_row_source(amk.AMK_ROLE_QKV, None, rows, 0) == -1
+    assert amk.amk_packed_row_source(amk.AMK_ROLE_PLAIN, None, 10, 10) == -1
+
+
+def test_step_bytes_model():
+    cfg = synth.preset("llama8b")
+    d = dims_of(cfg)
+    b = amk.amk_step_bytes(C.byref(d), 1023)
+    L, dm, ffn, V = 32, 4096, 14336, 128256
+    w = L * ((6144 + 4096) * dm + 2 * ffn * dm + dm * ffn) + V * dm
+    scales = 2 * (L * (6144 + dm + 2 * ffn + dm) + V)
+    kv = 2 * L * 8 * 1024 * 128 * 2
+    assert b == w + scales + dm * 2 + (2 * L + 1) * dm * 2 + kv
+    assert 7.5e9 < b < 7.8e9
+    d.weight_dtype = amk.AMK_W_BF16
+    assert amk.amk_step_bytes(C.byref(d), 1023) > 1.9 * b
+    assert amk.amk_step_bytes(None, 0) == 0
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+@pytest.mark.parametrize("grid", [148, 132, 16, 3])
+def test_plan_accepted(name, grid):
+    rc, msg = amk.plan_check(dims_of(synth.preset(name)), grid)
+    assert rc == amk.AMK_OK, msg
+
+
+@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("name", ["tiny", "llama8b"])
+def test_plan_defects_rejected(name, mutation):
+    rc, msg = amk.plan_check(dims_of(synth.preset(name)), 148, mutation)
+    assert rc == amk.AMK_ERR_PLAN, msg
+    assert msg and msg != "ok"
+
+
+def test_unsupported_dims_rejected():
+    d = dims_of(synth.preset("tiny"))
+    d.head_dim = 96
+    assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
+    d = dims_of(synth.preset("tiny"))
+    d.n_q_heads = 16          # group of 8
+    assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
+    d = dims_of(synth.preset("tiny"))
+    d.ffn = 700
+    assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
+    d = dims_of(synth.preset("tiny"))
+    d.n_layers = 0
+    assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_INVALID_ARG
+
+
+def test_argument_errors_before_any_launch():
+    h = C.c_void_p()
+    assert amk.amk_create(None, None, None, C.byref(h)) == amk.AMK_ERR_INVALID_ARG
+    assert amk.amk_create(None, None, None, None) == amk.AMK_ERR_INVALID_ARG
+    assert amk.amk_decode_step(None, 0, 0, None, None, None) == amk.AMK_ERR_INVALID_ARG
+    assert amk.amk_decode_step_unfused(None, 0, 0, None, None, None) == amk.AMK_ERR_INVALID_ARG
+    assert amk.amk_status(None, None) == amk.AMK_ERR_INVALID_ARG
+    d = dims_of(synth.preset("tiny"))
+    assert amk.amk_pack_weight(amk.AMK_ROLE_QKV, C.byref(d), None, 0, 512, 256, 0, None, None, None) == amk.AMK_ERR_INVALID_ARG
+    # wrong shape for the role is rejected on the host
+    assert amk.amk_pack_weight(amk.AMK_ROLE_QKV, C.byref(d), 16, 0, 100, 256, 0, 16, 16, None) == amk.AMK_ERR_INVALID_ARG
+    assert amk.amk_pack_weight(amk.AMK_ROLE_PLAIN, None, 16, 0, 4, 4, 0, 16, None, None) == amk.AMK_ERR_INVALID_ARG
+    assert amk.amk_trace_read(None, None, 0) == amk.AMK_ERR_INVALID_ARG
