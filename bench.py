@@ -101,53 +101,70 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 # CPU baseline: the oracle as it stands on a bounded sample of the workload
 
-def oracle_sample(cfg, reps: int = 1):
-    """Times oracle decode steps of the same shape with 1 and 2 layers; a full token costs
-    t(1 layer) + (L - 1) * (t(2 layers) - t(1 layer)). Returns (tokens/s, seconds measured, sample text)."""
-    import torch
-    from oracle import llama_decode as O
-    threads = torch.get_num_threads()
-    times = {}
+class OracleSample:
+    """The oracle as it stands, on a bounded sample of the workload: decode steps of models with the
+    same dims but 1 and 2 layers (same KV length). A full token costs t1 + (L - 1) * (t2 - t1)."""
+
+    def __init__(self, cfg):
+        import torch
+        from oracle import llama_decode as O
+        self.O = O
+        self.cfg = cfg
+        self.threads = torch.get_num_threads()
+        self.models = {}
+        for nl in (1, 2):
+            c = cfg.with_(n_layers=nl)
+            om = O.OracleModel(c, keep_dequantized=False)
+            kv = O.OracleKV(c, max_seq=c.prefill_len + c.prompt_len + 2)
+            kv.prefill_synthetic()
+            self.models[nl] = (om, kv, c.prefill_len + c.prompt_len)
+
+    def step(self, nl: int) -> float:
+        om, kv, pos = self.models[nl]
+        t0 = time.perf_counter()
+        self.O.decode_step(om, kv, 1, pos)
+        return time.perf_counter() - t0
+
+    def describe(self, n_timed: int) -> str:
+        c = self.cfg
+        return (f"oracle decode_step (torch CPU fp32, {self.threads} threads) on {c.name}-shaped models with 1 and 2 "
+                f"layers at KV length {c.prefill_len + c.prompt_len}; {n_timed} timed step(s); per-token time "
+                f"extrapolated to {c.n_layers} layers as t1 + {c.n_layers - 1}*(t2 - t1)")
+
+
+def oracle_tokens_per_s(cfg, reps: int = 3):
     t_all = time.time()
-    for nl in (1, 2):
-        c = cfg.with_(n_layers=nl, prefill_len=min(cfg.prefill_len, 1024))
-        om = O.OracleModel(c, keep_dequantized=False)
-        kv = O.OracleKV(c, max_seq=c.prefill_len + reps + 1)
-        kv.prefill_synthetic()
-        O.decode_step(om, kv, 1, c.prefill_len)            # warm-up
-        ts = []
-        for r in range(reps):
-            t0 = time.perf_counter()
-            O.decode_step(om, kv, 1 + r, c.prefill_len + r)
-            ts.append(time.perf_counter() - t0)
-        times[nl] = min(ts)
-        del om, kv
-    t_layer = max(times[2] - times[1], 0.0)
-    t_token = times[1] + (cfg.n_layers - 1) * t_layer
-    sample = (f"oracle decode_step on {cfg.name}-shaped models with 1 and 2 layers (same dims, same KV length "
-              f"{cfg.prefill_len}), {reps} timed step(s) each after 1 warm-up; per-token time extrapolated to "
-              f"{cfg.n_layers} layers as t1 + {cfg.n_layers - 1}*(t2 - t1)")
-    return 1.0 / t_token, time.time() - t_all, sample, threads
+    smp = OracleSample(cfg)
+    smp.step(1), smp.step(2)                               # warm-up
+    t1 = min(smp.step(1) for _ in range(reps))
+    t2 = min(smp.step(2) for _ in range(reps))
+    t_token = t1 + (cfg.n_layers - 1) * max(t2 - t1, 0.0)
+    return 1.0 / t_token, time.time() - t_all, smp.describe(2 * reps), smp.threads
 
 
 # ------------------------------------------------------------------------------------------------
 
 def run_reference(args, cfg, rank, world):
+    """The reference arm: the CPU oracle. Warm-up steps calibrate the per-layer cost (2-layer minus
+    1-layer step); each timed step is one 1-layer decode step; the reported rate is per full token."""
     if rank != 0:
         return
-    tps_list = []
-    cores = None
-    sample = ""
-    for i in range(args.warmup + args.steps):
-        tps, _, sample, cores = oracle_sample(cfg)
-        if i >= args.warmup:
-            tps_list.append(tps)
-    value = statistics.median(tps_list)
+    smp = OracleSample(cfg)
+    t1s, t2s = [], []
+    for _ in range(args.warmup):
+        t1s.append(smp.step(1))
+        t2s.append(smp.step(2))
+    t_layer = max(statistics.median(t2s) - statistics.median(t1s), 0.0)
+    timed = [smp.step(1) for _ in range(args.steps)]
+    t1 = statistics.median(timed)
+    value = 1.0 / (t1 + (cfg.n_layers - 1) * t_layer)
+    sample = smp.describe(args.steps) + "; per-layer cost calibrated over the warm-up steps"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": _workload_name(cfg)},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -287,7 +304,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, secs, sample, cores = oracle_sample(cfg)
+        tps, secs, sample, cores = oracle_tokens_per_s(cfg)
         cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(secs, 1)}
 
