@@ -74,6 +74,8 @@ amk_destroy = _sig("amk_destroy", None, C.c_void_p)
 amk_decode_step = _sig("amk_decode_step", C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p)
 amk_decode_step_unfused = _sig("amk_decode_step_unfused", C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
                                C.c_void_p, C.c_void_p)
+amk_decode_step_noalloc = _sig("amk_decode_step_noalloc", C.c_int, C.POINTER(amk_dims), C.POINTER(amk_weights),
+                               C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p)
 amk_status = _sig("amk_status", C.c_int, C.c_void_p, C.POINTER(C.c_uint32))
 amk_last_cuda_error = _sig("amk_last_cuda_error", C.c_char_p)
 amk_plan_info_get = _sig("amk_plan_info_get", C.c_int, C.c_void_p, C.POINTER(amk_plan_info))

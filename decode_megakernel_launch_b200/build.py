@@ -6,7 +6,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libamk.so")
-SOURCES = ["csrc/amk_device.cu", "csrc/amk_api.cu", "csrc/amk_plan.cpp"]
+SOURCES = ["csrc/amk_device.cu", "csrc/amk_api.cu", "csrc/amk_plan.cpp", "csrc/amk_noalloc.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 
 

@@ -39,6 +39,7 @@ extern "C" {
 #define AMK_ERR_UNSUPPORTED     -5  /* dims outside what the kernels support (see amk_create) */
 #define AMK_ERR_PLAN            -6  /* the static task-list check rejected the plan */
 #define AMK_ERR_NO_MEMORY       -7  /* host or device allocation failed */
+#define AMK_ERR_SCRATCH_LIMIT   -8  /* amk_decode_step_noalloc: dims need more than its fixed scratch */
 
 /* ---- enums ----------------------------------------------------------------------------------- */
 #define AMK_W_INT8   0   /* int8 weights, one bf16 scale per output row (W8A16) */
@@ -169,6 +170,32 @@ int  amk_status(const amk_handle* h, uint32_t* detail);
 
 /* Last CUDA error string seen by this library on this thread ("" if none). */
 const char* amk_last_cuda_error(void);
+
+/* ---- decode without device allocation ------------------------------------------------------- */
+
+/* The pages have no counterpart to this call; it is an interface addition of this library.
+ * Some callers can't call cudaMalloc: a plugin inside a host framework whose memory pool owns all of
+ * the device memory (an outside allocation fails near the pool's limit or is forbidden by policy), or a
+ * latency-critical loop where cudaMalloc/cudaFree may synchronize the whole device. amk_create
+ * allocates device state, so for them this call does the work of amk_create + amk_decode_step without
+ * allocating any device memory: the handle's state (task list, layer pointers, RoPE table, scratch
+ * vectors, attention partials, counters) lives in one static device array of 4 MiB inside libamk,
+ * resident on every GPU that loads the library until the process exits. It launches the same
+ * persistent kernel on the same plan (one CTA per SM, default options) as amk_decode_step.
+ *   dims, weights:  as for amk_create (same checks, same ownership: the caller owns every buffer).
+ *   token_id, pos, logits_out, next_token_out, stream: as for amk_decode_step.
+ * Returns AMK_ERR_SCRATCH_LIMIT, before launching anything, when the dims need more than 4 MiB of state
+ * (the task list grows with layers x SMs, the RoPE table with max_seq x head_dim: the 8B-shaped model
+ * with 1152 positions needs ~1.8 MiB). The first call on a device (with that device current) looks up
+ * the array's device address (cudaGetSymbolAddress) and sets the kernel's attributes; make that first
+ * call before any stream capture. Every call shares the array, which keeps the last call's contents:
+ * each call zeroes the counters and status words on `stream` and re-uploads the task list, layer
+ * pointers and RoPE table when dims or pointers differ from the previous call on that device. Calls
+ * whose launches overlap on the GPU (unordered streams) race on the array and must be serialized by
+ * the caller. A wait that expires inside such a launch is not reported (use amk_decode_step and
+ * amk_status for the sticky status). */
+int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* weights, int token_id, int pos,
+                            float* logits_out, int* next_token_out, void* stream);
 
 /* ---- plan introspection (host-only) ---------------------------------------------------------- */
 
