@@ -365,11 +365,15 @@ def main():
     ap.add_argument("--impl", default="amk", choices=["amk", "reference"])
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (smaller cases for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from decode_megakernel_launch_b200 import synth
     cfg = synth.preset(args.config)
+    if args.layers:
+        cfg = cfg.with_(n_layers=args.layers, name=f"{cfg.name}-{args.layers}layers")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -83,16 +83,6 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-// acc0 += lo(w) * lo(a); acc1 += hi(w) * hi(a)   (f16 x f16 -> f32, one rounding each)
-__device__ __forceinline__ void fma2_f16_f32(float& acc0, float& acc1, uint32_t w, uint32_t a) {
-  asm("{\n\t.reg .f16 w0, w1, a0, a1;\n\t"
-      "mov.b32 {w0, w1}, %2;\n\t"
-      "mov.b32 {a0, a1}, %3;\n\t"
-      "fma.rn.f32.f16 %0, w0, a0, %0;\n\t"
-      "fma.rn.f32.f16 %1, w1, a1, %1;\n\t}"
-      : "+f"(acc0), "+f"(acc1)
-      : "r"(w), "r"(a));
-}
 // acc += {lo, hi} * {a0, a1} with one packed fp32 FMA
 __device__ __forceinline__ void ffma2(unsigned long long& acc, float lo, float hi, float a0, float a1) {
   asm("{\n\t.reg .b64 wv, av;\n\t"
@@ -231,50 +221,122 @@ __device__ __forceinline__ bool is_gemv(int op) { return op == OP_QKV || op == O
 // ------------------------------------------------------------------------------------------------
 // Producer
 
-__device__ void producer(const Params& p, const Task* tasks, int nt, Smem& s) {
-  const uint64_t pol = policy_evict_first();
-  uint32_t it = 0;
-  auto acquire_slot = [&](uint32_t i) -> int {
-    const int slot = i % kSlots;
-    if (i >= (uint32_t)kSlots) wait_slot(p, &s.empty[slot], ((i / kSlots) - 1) & 1, (3u << 16) | slot);
-    return slot;
-  };
-  for (int ti = 0; ti < nt; ++ti) {
-    const Task t = tasks[ti];
-    if (is_gemv(t.op)) {
-      const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
-      const uint8_t* w = static_cast<const uint8_t*>(gemv_weights(p, t.op, t.layer));
-      for (int r = 0; r < t.b; r += g.rs, ++it) {
-        const int n = min(g.rs, t.b - r);
-        const int slot = acquire_slot(it);
-        const uint32_t bytes = (uint32_t)n * (uint32_t)g.rb;
-        mbar_expect_tx(&s.full[slot], bytes);
-        bulk_g2s(s.ring + slot * kSlotBytes, w + (size_t)(t.a + r) * g.rb, bytes, &s.full[slot], pol);
-      }
-    } else if (t.op == OP_ATTN) {
-      const int P = p.pos + 1;
-      const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
-      if (t.b >= C) continue;
-      int cb, ce;
-      attn_chunk_range(P, C, t.b, &cb, &ce);
-      const int nps = attn_positions_per_slot(p.hd);
-      const size_t row_bytes = (size_t)p.hd * 2;
-      const size_t head_off = ((size_t)t.layer * p.Hkv + t.a) * p.max_seq;
-      for (int blk = cb; blk < ce; blk += nps, ++it) {
-        const int be = min(blk + nps, ce);
-        const int ntma = min(be, p.pos) - blk;   // row `pos` is written this step: patched in smem
-        const int slot = acquire_slot(it);
-        if (ntma > 0) {
-          const uint32_t bytes = (uint32_t)(ntma * row_bytes);
-          mbar_expect_tx(&s.full[slot], 2 * bytes);
-          uint8_t* dst = s.ring + slot * kSlotBytes;
-          bulk_g2s(dst, p.kcache + (head_off + blk) * p.hd, bytes, &s.full[slot], pol);
-          bulk_g2s(dst + kSlotBytes / 2, p.vcache + (head_off + blk) * p.hd, bytes, &s.full[slot], pol);
-        } else {
-          mbar_arrive(&s.full[slot]);
-        }
+// Walks the byte stream of one CTA's task list, one ring slot (item) at a time. An item is one
+// contiguous weight range (GEMV rows) or a K range plus the matching V range (attention).
+struct ItemCursor {
+  int ti = 0;       // task index
+  int sub = 0;      // GEMV: first row of the item; ATTN: first position of the item
+  bool started = false;
+  int end = 0;      // GEMV: rows; ATTN: chunk end position
+};
+
+// Advances `c` to the next item; returns false at the end of the list. (src0, n0) and (src1, n1)
+// are the item's byte ranges (n1 = 0 for GEMV items; n0 = n1 = 0 for an attention block that holds
+// only the current position, which is written this step and patched in shared memory).
+__device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor& c, const uint8_t*& src0,
+                          uint32_t& n0, const uint8_t*& src1, uint32_t& n1) {
+  while (c.ti < nt) {
+    const Task& t = tasks[c.ti];
+    if (!c.started) {
+      c.started = true;
+      if (t.op == OP_ATTN) {
+        const int P = p.pos + 1;
+        const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
+        int cb = 0, ce = 0;
+        if (t.b < C) attn_chunk_range(P, C, t.b, &cb, &ce);
+        c.sub = cb;
+        c.end = ce;
+      } else if (is_gemv(t.op)) {
+        c.sub = 0;
+        c.end = t.b;
+      } else {
+        c.sub = c.end = 0;
       }
     }
+    if (c.sub < c.end) {
+      if (t.op == OP_ATTN) {
+        const int nps = attn_positions_per_slot(p.hd);
+        const int blk = c.sub, be = min(blk + nps, c.end);
+        const int ntma = max(0, min(be, p.pos) - blk);
+        const size_t off = (((size_t)t.layer * p.Hkv + t.a) * p.max_seq + blk) * p.hd;
+        src0 = reinterpret_cast<const uint8_t*>(p.kcache + off);
+        src1 = reinterpret_cast<const uint8_t*>(p.vcache + off);
+        n0 = n1 = (uint32_t)ntma * (uint32_t)p.hd * 2u;
+        c.sub = be;
+      } else {
+        const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
+        const int n = min(g.rs, c.end - c.sub);
+        src0 = static_cast<const uint8_t*>(gemv_weights(p, t.op, t.layer)) + (size_t)(t.a + c.sub) * g.rb;
+        n0 = (uint32_t)n * (uint32_t)g.rb;
+        src1 = nullptr;
+        n1 = 0;
+        c.sub += n;
+      }
+      return true;
+    }
+    ++c.ti;
+    c.started = false;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void prefetch_line_l2(const void* a) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a) : "memory");
+}
+__device__ __forceinline__ void prefetch_bulk_l2(const void* a, uint32_t bytes) {   // 16-B aligned, 16-B multiple
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(bytes) : "memory");
+}
+
+// L2 prefetch of the small static data a task reads on its critical path (row scales, RMSNorm gain,
+// this position's RoPE row, the embedding row), issued when the producer starts streaming the
+// task's weights, i.e. several ring slots before the compute warps reach it. Under a full HBM
+// stream an L2 miss costs microseconds, so these would otherwise stall every stage transition.
+__device__ void prefetch_side_data(const Params& p, const Task& t, int token) {
+  if (!is_gemv(t.op)) return;
+  const uint16_t* sc = gemv_scales(p, t.op, t.layer);
+  if (p.wdtype == AMK_W_INT8 && sc && t.b > 0) {
+    const char* b = reinterpret_cast<const char*>(sc + t.a);
+    const int bytes = t.b * 2;
+    for (int o = 0; o < bytes; o += 128) prefetch_line_l2(b + o);
+    prefetch_line_l2(b + bytes - 1);
+  }
+  const uint16_t* gain = t.op == OP_QKV ? p.layers[t.layer].attn_norm
+                       : t.op == OP_GU ? p.layers[t.layer].ffn_norm
+                       : t.op == OP_LM ? p.final_norm : nullptr;
+  if (gain) prefetch_bulk_l2(gain, (uint32_t)p.d * 2);
+  if (t.op == OP_QKV) {
+    prefetch_bulk_l2(p.rope + (size_t)p.pos * p.hd, (uint32_t)p.hd * 4);
+    if (t.layer == 0) prefetch_bulk_l2(p.embed + (size_t)token * p.d, (uint32_t)p.d * 2);
+  }
+}
+
+// Producer lane: issues every item of the CTA's byte stream into the ring in order, gated only by
+// the ring's empty barriers (never by other CTAs).
+__device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt, Smem& s) {
+  const uint64_t pol = policy_evict_first();
+  int token = p.token;
+  if (token < 0) token = __ldcg(p.next_token);
+  if (token < 0 || token >= p.V) token = 0;
+  ItemCursor cur;
+  uint32_t it = 0;
+  int last_task = -1;
+  const uint8_t *a0, *a1;
+  uint32_t n0, n1;
+  while (next_item(p, tasks, nt, cur, a0, n0, a1, n1)) {
+    if (cur.ti != last_task) {
+      last_task = cur.ti;
+      prefetch_side_data(p, tasks[cur.ti], token);
+    }
+    const int slot = it % kSlots;
+    if (it >= (uint32_t)kSlots) wait_slot(p, &s.empty[slot], ((it / kSlots) - 1) & 1, (3u << 16) | slot);
+    if (n0 + n1 > 0) {
+      mbar_expect_tx(&s.full[slot], n0 + n1);
+      bulk_g2s(s.ring + slot * kSlotBytes, a0, n0, &s.full[slot], pol);
+      if (n1) bulk_g2s(s.ring + slot * kSlotBytes + kSlotBytes / 2, a1, n1, &s.full[slot], pol);
+    } else {
+      mbar_arrive(&s.full[slot]);
+    }
+    ++it;
   }
 }
 
@@ -313,16 +375,34 @@ __device__ __forceinline__ float reduce4_rows(float a0, float a1, float a2, floa
   return u;
 }
 
+// Sum of 2 per-lane values for 2 rows over the warp; lanes 0..15 return row 0's total and lanes
+// 16..31 row 1's (transposed butterfly: 5 shuffles for 2 rows).
+__device__ __forceinline__ float reduce2_rows(float a0, float a1) {
+  const int lane = threadIdx.x & 31;
+  const bool u16 = lane & 16;
+  float k = u16 ? a1 : a0;
+  k += __shfl_xor_sync(0xffffffffu, u16 ? a0 : a1, 16);
+  k += __shfl_xor_sync(0xffffffffu, k, 8);
+  k += __shfl_xor_sync(0xffffffffu, k, 4);
+  k += __shfl_xor_sync(0xffffffffu, k, 2);
+  k += __shfl_xor_sync(0xffffffffu, k, 1);
+  return k;
+}
+
 template <int GB>
 struct GroupWords { static constexpr int N = GB >= 4 ? GB / 4 : 1; };
 
+// One thread's group of GB weight bytes of a row: 16-byte vector loads (GB >= 16) or one smaller one.
 template <int GB>
 __device__ __forceinline__ void lds_group(const uint8_t* ptr, uint32_t (&w)[GroupWords<GB>::N]) {
-  if constexpr (GB == 16) {
-    uint4 v = *reinterpret_cast<const uint4*>(ptr);
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  if constexpr (GB >= 16) {
+#pragma unroll
+    for (int i = 0; i < GB / 16; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(ptr)[i];
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
   } else if constexpr (GB == 8) {
-    uint2 v = *reinterpret_cast<const uint2*>(ptr);
+    const uint2 v = *reinterpret_cast<const uint2*>(ptr);
     w[0] = v.x; w[1] = v.y;
   } else if constexpr (GB == 4) {
     w[0] = *reinterpret_cast<const uint32_t*>(ptr);
@@ -331,119 +411,176 @@ __device__ __forceinline__ void lds_group(const uint8_t* ptr, uint32_t (&w)[Grou
   }
 }
 
-// int8 group against f16 activations: acc += sum_e (q_e + 1152) * a_e  (the +1152 is removed later
-// with the thread's activation sum). Each int8 byte becomes the f16 1024 + (q ^ 0x80) exactly.
-template <int GB>
-__device__ __forceinline__ void dot_i8(float& acc0, float& acc1, const uint32_t (&w)[GroupWords<GB>::N],
-                                       const uint32_t* a) {
-  if constexpr (GB >= 4) {
+// int8 chunk of ECH elements against int16 activations: exact int32 dot product with dp2a (two
+// int16 x int8 products per instruction; .lo takes weight bytes 0-1, .hi bytes 2-3). Activation word k
+// holds elements 2k (low half) and 2k+1 (high half).
+template <int ECH>
+__device__ __forceinline__ int dot_chunk_i8(int acc, const uint32_t* w, const uint32_t* a) {
+  if constexpr (ECH >= 4) {
 #pragma unroll
-    for (int k = 0; k < GB / 4; ++k) {
-      const uint32_t x = w[k] ^ 0x80808080u;
-      const uint32_t h01 = __byte_perm(x, 0x64646464u, 0x4140);
-      const uint32_t h23 = __byte_perm(x, 0x64646464u, 0x4342);
-      fma2_f16_f32(acc0, acc1, h01, a[2 * k]);
-      fma2_f16_f32(acc0, acc1, h23, a[2 * k + 1]);
+    for (int k = 0; k < ECH / 4; ++k) {
+      acc = __dp2a_lo((int)a[2 * k], (int)w[k], acc);
+      acc = __dp2a_hi((int)a[2 * k + 1], (int)w[k], acc);
     }
   } else {
-    const uint32_t x = w[0] ^ 0x8080u;
-    const uint32_t h01 = __byte_perm(x, 0x64646464u, 0x4140);
-    fma2_f16_f32(acc0, acc1, h01, a[0]);
+    acc = __dp2a_lo((int)a[0], (int)w[0], acc);
   }
+  return acc;
 }
 
-// bf16 group against fp32 activations (packed fp32 FMAs).
-template <int GB>
-__device__ __forceinline__ void dot_bf16(unsigned long long& acc, const uint32_t (&w)[GroupWords<GB>::N],
-                                         const float* a) {
+// Vector loads of N consecutive elements (N in {2, 4, 8, 16}) into fp32 registers.
+template <int N>
+__device__ __forceinline__ void ld_f32_cg(const float* p, float* o) {   // written by other CTAs: L2 only
+  if constexpr (N >= 4) {
 #pragma unroll
-  for (int k = 0; k < GB / 4; ++k) {
-    const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xffff0000u);
-    ffma2(acc, lo, hi, a[2 * k], a[2 * k + 1]);
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + i);
+      o[4 * i] = v.x; o[4 * i + 1] = v.y; o[4 * i + 2] = v.z; o[4 * i + 3] = v.w;
+    }
+  } else {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p));
+    o[0] = v.x; o[1] = v.y;
   }
 }
+template <int N>
+__device__ __forceinline__ void ld_bf16_words(const uint16_t* p, uint32_t* o) {   // read-only: N/2 words
+  if constexpr (N >= 8) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + i);
+      o[4 * i] = v.x; o[4 * i + 1] = v.y; o[4 * i + 2] = v.z; o[4 * i + 3] = v.w;
+    }
+  } else if constexpr (N == 4) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    o[0] = v.x; o[1] = v.y;
+  } else {
+    o[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
+  }
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Source vector element `e` of the GEMV of `op` (before the f16 / fp32 packing).
-struct VecSrc {
-  const float* f32;       // x / attn_out / act, or null
-  const uint16_t* bf16;   // embedding row (first QKV), or null
-  const uint16_t* gain;   // RMSNorm gain, or null
-  float inv;              // 1 / rms, or 1
-};
-
-__device__ __forceinline__ float vec_elem(const VecSrc& v, int e) {
-  float x = v.f32 ? __ldcg(v.f32 + e) : bf2f(v.bf16[e]);
-  if (v.gain) x = x * v.inv * bf2f(v.gain[e]);
-  return x;
+// Byte offset, inside a row, of piece c of the group that (warp column col, lane) owns. A group of
+// GB bytes is min(GB, 16)-byte pieces laid 32 pieces apart, so one load instruction of a warp reads
+// 32 x 16 contiguous bytes (no shared-memory bank conflicts).
+template <int GB>
+__device__ __forceinline__ int piece_offset(int col, int lane, int c) {
+  constexpr int PB = GB < 16 ? GB : 16;
+  return col * 32 * GB + c * 32 * PB + lane * PB;
 }
 
-template <bool I8, int GB>
-__device__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it, int token) {
-  constexpr int NRMAX = (I8 ? 32 : 64) / GB;             // 16 f16x2 or 32 fp32 activation registers
-  constexpr int EPG = I8 ? GB : GB / 2;                 // elements per group
-  constexpr int AW = I8 ? (GB >= 4 ? GB / 2 : 1) : EPG; // activation registers per group
+// One GEMV task: rows [t.a, t.a + t.b) of the op's packed matrix against this step's input vector.
+// I8: int8 weights, dp2a against int16 activations quantised per 16-byte piece; otherwise bf16
+// weights with packed fp32 FMAs. GB: weight bytes per thread per row; NR: compile-time bound on
+// groups per thread (geometry nr <= NR). For RMSNorm inputs the thread works on x * g and the
+// 1/rms factor is applied per row in the epilogue, so the input loads need one L2 round trip.
+template <bool I8, int GB, int NR>
+__device__ __noinline__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it, int token,
+                          unsigned long long* tr) {
+  constexpr int ES = I8 ? 1 : 2;                        // weight element bytes
+  constexpr int PB = GB < 16 ? GB : 16;                 // bytes per piece
+  constexpr int NP = GB / PB;                           // pieces per group
+  constexpr int PE = PB / ES;                           // elements per piece
+  constexpr int NB = GB >= 64 ? 1 : GB >= 32 ? 2 : 4;   // rows per register batch
+  constexpr int WPP = PB >= 4 ? PB / 4 : 1;             // weight words per piece
   const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int op = t.op, l = t.layer, row0 = t.a, nrows = t.b;
   const bool first = t.flags & kFirstOfStage;
+  const int rp = warp / g.wpg, wg = warp % g.wpg;
+  const bool active = rp < g.rp;
+  const bool norm = op == OP_QKV || op == OP_GU || op == OP_LM;
 
+  // ---- static data first (scales), so its latency hides behind the wait ----
   const uint16_t* sc = I8 ? gemv_scales(p, op, l) : nullptr;
   if (I8 && sc)
     for (int i = tid; i < nrows; i += kConsumerThreads) s.scale[i] = bf2f(__ldg(sc + row0 + i));
+  bool ok[NR];
+  int col[NR];
+#pragma unroll
+  for (int j = 0; j < NR; ++j) {
+    col[j] = j * g.wpg + wg;
+    ok[j] = active && j < g.nr && col[j] < g.wg_total;
+  }
 
   if (p.sync && first && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
+  if (tr && tid == 0) tr[2] = globaltimer();
 
-  // ---- activations of this thread's groups (kept in registers for the whole task) ----
-  VecSrc v{nullptr, nullptr, nullptr, 1.f};
-  if (op == OP_QKV || op == OP_GU || op == OP_LM) {
-    if (op == OP_QKV && l == 0) v.bf16 = p.embed + (size_t)token * p.d;
-    else v.f32 = p.x;
-    v.gain = op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : p.final_norm;
-    float ss = 0.f;
-    for (int e = tid; e < p.d; e += kConsumerThreads) {
-      const float x = v.f32 ? __ldcg(v.f32 + e) : bf2f(v.bf16[e]);
-      ss += x * x;
-    }
-    ss = block_sum(ss, s);
-    v.inv = rsqrtf(ss / (float)p.d + p.eps);
-  } else {
-    v.f32 = op == OP_O ? p.attn_out : p.act;
-  }
-
-  const int rp = warp / g.wpg, wg = warp % g.wpg;
-  const bool active = rp < g.rp;
-  uint32_t ah[I8 ? NRMAX * AW : 1];
-  float af[I8 ? 1 : NRMAX * AW];
-  float asum = 0.f;
-#pragma unroll
-  for (int j = 0; j < NRMAX; ++j) {
-    const int col = j * g.wpg + wg;
-    const bool ok = active && j < g.nr && col < g.wg_total;
-    const int e0 = (col * 32 + lane) * EPG;
-    if constexpr (I8) {
-#pragma unroll
-      for (int k = 0; k < AW; ++k) {
-        float x0 = 0.f, x1 = 0.f;
-        if (ok) {
-          x0 = vec_elem(v, e0 + 2 * k);
-          if (EPG > 1) x1 = vec_elem(v, e0 + 2 * k + 1);
-        }
-        __half2 h = __floats2half2_rn(x0, x1);
-        asum += __low2float(h) + __high2float(h);
-        ah[j * AW + k] = *reinterpret_cast<uint32_t*>(&h);
+  // ---- inputs: the RMS pass (coalesced) and this thread's own elements, all loads in flight ----
+  const bool from_embed = op == OP_QKV && l == 0;
+  const float* src = op == OP_O ? p.attn_out : op == OP_DOWN ? p.act : p.x;
+  const uint16_t* erow = p.embed + (size_t)token * p.d;
+  const uint16_t* gain =
+      op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : op == OP_LM ? p.final_norm : nullptr;
+  float ss = 0.f;
+  if (norm) {
+    for (int e = tid * 4; e < p.d; e += kConsumerThreads * 4) {
+      float v[4];
+      if (from_embed) {
+        uint32_t w2[2];
+        ld_bf16_words<4>(erow + e, w2);
+        v[0] = bf_lo(w2[0]); v[1] = bf_hi(w2[0]); v[2] = bf_lo(w2[1]); v[3] = bf_hi(w2[1]);
+      } else {
+        ld_f32_cg<4>(src + e, v);
       }
-    } else {
-#pragma unroll
-      for (int k = 0; k < AW; ++k) af[j * AW + k] = ok ? vec_elem(v, e0 + k) : 0.f;
+      ss = fmaf(v[0], v[0], fmaf(v[1], v[1], fmaf(v[2], v[2], fmaf(v[3], v[3], ss))));
     }
   }
-  const float corr = 1152.f * asum;
+  float xv[NR * NP * PE];
+#pragma unroll
+  for (int j = 0; j < NR; ++j) {
+#pragma unroll
+    for (int c = 0; c < NP; ++c) {
+      float* xp = &xv[(j * NP + c) * PE];
+      const int e = piece_offset<GB>(col[j], lane, c) / ES;
+      if (ok[j]) {
+        if (from_embed) {
+          uint32_t ew[PE / 2];
+          ld_bf16_words<PE>(erow + e, ew);
+#pragma unroll
+          for (int k = 0; k < PE / 2; ++k) { xp[2 * k] = bf_lo(ew[k]); xp[2 * k + 1] = bf_hi(ew[k]); }
+        } else {
+          ld_f32_cg<PE>(src + e, xp);
+        }
+        if (norm) {
+          uint32_t gw[PE / 2];
+          ld_bf16_words<PE>(gain + e, gw);
+#pragma unroll
+          for (int k = 0; k < PE / 2; ++k) { xp[2 * k] *= bf_lo(gw[k]); xp[2 * k + 1] *= bf_hi(gw[k]); }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < PE; ++k) xp[k] = 0.f;
+      }
+    }
+  }
+  float inv = 1.f;
+  if (norm) inv = rsqrtf(block_sum(ss, s) / (float)p.d + p.eps);
+
+  uint32_t ah[I8 ? NR * NP * PE / 2 : 1];
+  float asc[I8 ? NR * NP : 1];   // per-piece scale: activation = int16 * asc
+  if constexpr (I8) {
+#pragma unroll
+    for (int c = 0; c < NR * NP; ++c) {
+      float amax = 0.f;
+#pragma unroll
+      for (int k = 0; k < PE; ++k) amax = fmaxf(amax, fabsf(xv[c * PE + k]));
+      const float q = amax > 0.f ? 32767.f / amax : 0.f;
+      asc[c] = amax * (1.f / 32767.f);
+#pragma unroll
+      for (int k = 0; k < PE / 2; ++k) {
+        const int lo = __float2int_rn(xv[c * PE + 2 * k] * q), hi = __float2int_rn(xv[c * PE + 2 * k + 1] * q);
+        ah[c * PE / 2 + k] = ((uint32_t)lo & 0xffffu) | ((uint32_t)hi << 16);
+      }
+    }
+  }
 
   // ---- rows, one ring slot at a time ----
   const int blk_rows = g.rs * (kRowBlock / g.rs);
   const int rpg = (g.rs + g.rp - 1) / g.rp;
   float lm_v = -CUDART_INF_F;
   int lm_i = 0x7fffffff;
+  int blk_base = 0;                         // task-relative first row of the current epilogue block
   for (int r0 = 0; r0 < nrows; r0 += g.rs, ++it) {
     const int slot = it % kSlots;
     wait_slot(p, &s.full[slot], (it / kSlots) & 1, (2u << 16) | slot);
@@ -451,31 +588,50 @@ __device__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it,
     const uint8_t* sbuf = s.ring + slot * kSlotBytes;
     if (active) {
       const int rb0 = rp * rpg, re = min(rb0 + rpg, srows);
-      for (int r = rb0; r < re; r += 4) {
-        float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-        unsigned long long accp[4] = {0ull, 0ull, 0ull, 0ull};
+      for (int r = rb0; r < re; r += NB) {
+        float a[NB];
 #pragma unroll
-        for (int j = 0; j < NRMAX; ++j) {
-          const int col = j * g.wpg + wg;
-          if (j < g.nr && col < g.wg_total) {
-            const int boff = (col * 32 + lane) * GB;
+        for (int rr = 0; rr < NB; ++rr) {
+          float v = 0.f;
+          if (r + rr < re) {
+            const uint8_t* rowp = sbuf + (size_t)(r + rr) * g.rb;
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-              if (r + rr < re) {
-                uint32_t w[GroupWords<GB>::N];
-                lds_group<GB>(sbuf + (size_t)(r + rr) * g.rb + boff, w);
-                if constexpr (I8) dot_i8<GB>(acc[rr][0], acc[rr][1], w, &ah[j * AW]);
-                else dot_bf16<GB>(accp[rr], w, &af[j * AW]);
+            for (int j = 0; j < NR; ++j) {
+              if (ok[j]) {
+#pragma unroll
+                for (int c = 0; c < NP; ++c) {
+                  uint32_t w[WPP];
+                  lds_group<PB>(rowp + piece_offset<GB>(col[j], lane, c), w);
+                  if constexpr (I8) {
+                    const int acc = dot_chunk_i8<PE>(0, w, &ah[(j * NP + c) * PE / 2]);
+                    v = fmaf((float)acc, asc[j * NP + c], v);
+                  } else {
+                    unsigned long long acc2 = 0ull;
+#pragma unroll
+                    for (int k = 0; k < WPP; ++k)
+                      ffma2(acc2, bf_lo(w[k]), bf_hi(w[k]), xv[(j * NP + c) * PE + 2 * k], xv[(j * NP + c) * PE + 2 * k + 1]);
+                    v += f2sum(acc2);
+                  }
+                }
               }
             }
           }
+          a[rr] = v;
         }
-        float a4[4];
+        if constexpr (NB == 1) {
+          float tot = a[0];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) a4[rr] = I8 ? (acc[rr][0] + acc[rr][1]) - corr : f2sum(accp[rr]);
-        const float tot = reduce4_rows(a4[0], a4[1], a4[2], a4[3]);
-        const int row = r + ((lane >> 3) & 3);
-        if ((lane & 7) == 0 && row < re) s.part[wg * kRowBlock + ((r0 + row) % blk_rows)] = tot;
+          for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+          if (lane == 0) s.part[wg * kRowBlock + (r0 + r - blk_base)] = tot;
+        } else if constexpr (NB == 2) {
+          const float tot = reduce2_rows(a[0], a[1]);
+          const int row = r + (lane >> 4);
+          if ((lane & 15) == 0 && row < re) s.part[wg * kRowBlock + (r0 + row - blk_base)] = tot;
+        } else {
+          const float tot = reduce4_rows(a[0], a[1], a[2], a[3]);
+          const int row = r + ((lane >> 3) & 3);
+          if ((lane & 7) == 0 && row < re) s.part[wg * kRowBlock + (r0 + row - blk_base)] = tot;
+        }
       }
     }
     __syncwarp();
@@ -483,13 +639,14 @@ __device__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it,
 
     // ---- epilogue of a finished block of rows ----
     const int done = r0 + srows;
-    if (done % blk_rows == 0 || done == nrows) {
+    if (done - blk_base == blk_rows || done == nrows) {
       bar_compute();
-      const int bs = ((done - 1) / blk_rows) * blk_rows, bn = done - bs;
+      const int bs = blk_base, bn = done - blk_base;
       auto rowsum = [&](int rr) {
-        float a = 0.f;
-        for (int w = 0; w < g.wpg; ++w) a += s.part[w * kRowBlock + rr];
-        return I8 && sc ? a * s.scale[bs + rr] : a;
+        float acc = 0.f;
+        for (int w = 0; w < g.wpg; ++w) acc += s.part[w * kRowBlock + rr];
+        acc *= inv;
+        return I8 && sc ? acc * s.scale[bs + rr] : acc;
       };
       if (op == OP_QKV || op == OP_GU) {
         for (int pr = tid; pr < bn / 2; pr += kConsumerThreads) {
@@ -531,6 +688,7 @@ __device__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it,
         }
       }
       bar_compute();
+      blk_base = done;
     }
   }
 
@@ -559,41 +717,84 @@ __device__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it,
   }
 }
 
+// Picks the register footprint: one group per thread, or the most the bytes per thread allow
+// (<= 32 int8 / 32 bf16 activations per thread).
+template <bool I8, int GB>
+__device__ __forceinline__ void gemv_nr(const Params& p, const Task& t, Smem& s, uint32_t& it, int token,
+                                        unsigned long long* tr, int nr) {
+  constexpr int NRMAX = (I8 ? 32 : 64) / GB;
+  if constexpr (NRMAX <= 1) {
+    gemv_task<I8, GB, 1>(p, t, s, it, token, tr);
+  } else {
+    if (nr <= 1) gemv_task<I8, GB, 1>(p, t, s, it, token, tr);
+    else gemv_task<I8, GB, NRMAX>(p, t, s, it, token, tr);
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Attention (split-KV flash decoding)
 
 __device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : exp2f(m - M); }
 
-// Log-sum-exp merge of the C chunk partials of KV head h into attn_out.
-__device__ void merge_head(const Params& p, int h, int C) {
+// Log-sum-exp merge of the C chunk partials of KV head h into attn_out. Chunks are read 16 at a time
+// with all their loads in flight, folded into a running (max, sum, output) per element.
+__device__ __noinline__ void merge_head(const Params& p, int h, int C) {
+  constexpr int B = 8;
   const int G = p.Hq / p.Hkv, hd = p.hd;
   const int stride = hd + 2;
   for (int idx = threadIdx.x; idx < G * hd; idx += kConsumerThreads) {
     const int g = idx / hd, e = idx % hd;
-    float M = -CUDART_INF_F;
-    for (int c = 0; c < C; ++c) {
-      const float* pc = p.attn_part + (((size_t)h * p.kv_chunks_max + c) * G + g) * stride;
-      M = fmaxf(M, __ldcg(pc + hd));
-    }
-    float Ls = 0.f, O = 0.f;
-    for (int c = 0; c < C; ++c) {
-      const float* pc = p.attn_part + (((size_t)h * p.kv_chunks_max + c) * G + g) * stride;
-      const float f = exp2_scale(__ldcg(pc + hd), M);
-      Ls += __ldcg(pc + hd + 1) * f;
-      O += __ldcg(pc + e) * f;
+    const float* base = p.attn_part + ((size_t)h * p.kv_chunks_max * G + g) * stride;
+    const size_t cstride = (size_t)G * stride;
+    float M = -CUDART_INF_F, Ls = 0.f, O = 0.f;
+    for (int c0 = 0; c0 < C; c0 += B) {
+      float mm[B], ll[B], oo[B];
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const bool v = c0 + i < C;
+        const float* pc = base + (size_t)(c0 + i) * cstride;
+        mm[i] = v ? __ldcg(pc + hd) : -CUDART_INF_F;
+        ll[i] = v ? __ldcg(pc + hd + 1) : 0.f;
+        oo[i] = v ? __ldcg(pc + e) : 0.f;
+      }
+      float Mn = M;
+#pragma unroll
+      for (int i = 0; i < B; ++i) Mn = fmaxf(Mn, mm[i]);
+      const float f = exp2_scale(M, Mn);
+      Ls *= f;
+      O *= f;
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const float fi = exp2_scale(mm[i], Mn);
+        Ls = fmaf(ll[i], fi, Ls);
+        O = fmaf(oo[i], fi, O);
+      }
+      M = Mn;
     }
     p.attn_out[(h * G + g) * hd + e] = O / Ls;
   }
 }
 
+// Split-KV flash decoding of one (KV head, chunk) task. The compute warps form NHG groups, one per
+// pair of query heads of this KV head's GQA group (kHeadsPerWarp = 2 keeps a warp's running state
+// small: 2 x (max, sum, 8 outputs) per lane). Inside a warp, LPP lanes hold one 16-byte piece of a
+// key/value row (8 elements) and PPW positions are processed per step; each sub-warp keeps an online
+// softmax, merged across sub-warps by shuffles and across the group's warps by a shared-memory tree.
+constexpr int kHeadsPerWarp = 2;
+
 template <int HD>
-__device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it) {
-  constexpr int LPP = HD * 2 / 16;       // lanes per position (one 16-byte chunk each)
+__device__ __noinline__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it, unsigned long long* tr) {
+  constexpr int LPP = HD * 2 / 16;       // lanes per position (one 16-byte piece each)
   constexpr int PPW = 32 / LPP;          // positions per warp step
   constexpr int NPS = kSlotBytes / (4 * HD);
+  constexpr int HW = kHeadsPerWarp;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cl = lane % LPP, sw = lane / LPP;
   const int G = p.Hq / p.Hkv;
+  const int NHG = (G + HW - 1) / HW;                 // head groups
+  const int WPH = kConsumerWarps / NHG;              // warps per head group (8 or 16)
+  const int hg = warp / WPH, wi = warp % WPH;
+  const bool in_group = hg < NHG;
   const int h = t.a, c = t.b, l = t.layer;
   const int P = p.pos + 1;
   const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
@@ -602,6 +803,7 @@ __device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it)
   attn_chunk_range(P, C, c, &cb, &ce);
 
   if (p.sync && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
+  if (tr && tid == 0) tr[2] = globaltimer();
 
   // queries of this KV head's group, pre-scaled by log2(e) / sqrt(hd), staged in shared memory
   // (the GEMV partial-sum region, which attention tasks do not use)
@@ -610,14 +812,15 @@ __device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it)
   for (int i = tid; i < G * HD; i += kConsumerThreads) qsm[i] = __ldcg(p.q + h * G * HD + i) * qs;
   bar_compute();
 
-  float m[kMaxGroup], ls[kMaxGroup], o[kMaxGroup][8];
+  float m[HW], ls[HW], o[HW][8];
 #pragma unroll
-  for (int g = 0; g < kMaxGroup; ++g) {
+  for (int g = 0; g < HW; ++g) {
     m[g] = -CUDART_INF_F;
     ls[g] = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
   }
+  const int g0 = hg * HW;                               // first query head of this warp's group
 
   const size_t head_off = ((size_t)l * p.Hkv + h) * p.max_seq;
   for (int blk = cb; blk < ce; blk += NPS, ++it) {
@@ -638,48 +841,50 @@ __device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it)
       }
       bar_compute();
     }
-    for (int base = 0; base < n; base += kConsumerWarps * PPW) {
-      const int j = base + warp * PPW + sw;
-      const bool valid = j < n;
-      float sc[kMaxGroup];
-      {
-        const uint4 kw = valid ? *reinterpret_cast<const uint4*>(kb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
-        const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+    if (in_group) {
+      for (int base = 0; base < n; base += WPH * PPW) {
+        const int j = base + wi * PPW + sw;
+        const bool valid = j < n;
+        float sc[HW];
+        {
+          const uint4 kw = valid ? *reinterpret_cast<const uint4*>(kb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
+          const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) {
-          float a = 0.f;
-          if (g < G) {
-            const float4 q0 = *reinterpret_cast<const float4*>(qsm + g * HD + cl * 8);
-            const float4 q1 = *reinterpret_cast<const float4*>(qsm + g * HD + cl * 8 + 4);
-            a = fmaf(q0.x, __uint_as_float(kk[0] << 16), a);
-            a = fmaf(q0.y, __uint_as_float(kk[0] & 0xffff0000u), a);
-            a = fmaf(q0.z, __uint_as_float(kk[1] << 16), a);
-            a = fmaf(q0.w, __uint_as_float(kk[1] & 0xffff0000u), a);
-            a = fmaf(q1.x, __uint_as_float(kk[2] << 16), a);
-            a = fmaf(q1.y, __uint_as_float(kk[2] & 0xffff0000u), a);
-            a = fmaf(q1.z, __uint_as_float(kk[3] << 16), a);
-            a = fmaf(q1.w, __uint_as_float(kk[3] & 0xffff0000u), a);
-          }
-#pragma unroll
-          for (int off = 1; off < LPP; off <<= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-          sc[g] = a;
-        }
-      }
-      if (valid) {
-        const uint4 vw = *reinterpret_cast<const uint4*>(vb + (size_t)j * HD * 2 + cl * 16);
-        const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) {
-          if (g < G) {
-            const float mn = fmaxf(m[g], sc[g]);
-            const float cr = exp2_scale(m[g], mn), pe = exp2f(sc[g] - mn);
-            ls[g] = ls[g] * cr + pe;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              o[g][2 * q] = fmaf(o[g][2 * q], cr, pe * __uint_as_float(vv[q] << 16));
-              o[g][2 * q + 1] = fmaf(o[g][2 * q + 1], cr, pe * __uint_as_float(vv[q] & 0xffff0000u));
+          for (int g = 0; g < HW; ++g) {
+            float a = 0.f;
+            if (g0 + g < G) {
+              const float4 q0 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8);
+              const float4 q1 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8 + 4);
+              a = fmaf(q0.x, bf_lo(kk[0]), a);
+              a = fmaf(q0.y, bf_hi(kk[0]), a);
+              a = fmaf(q0.z, bf_lo(kk[1]), a);
+              a = fmaf(q0.w, bf_hi(kk[1]), a);
+              a = fmaf(q1.x, bf_lo(kk[2]), a);
+              a = fmaf(q1.y, bf_hi(kk[2]), a);
+              a = fmaf(q1.z, bf_lo(kk[3]), a);
+              a = fmaf(q1.w, bf_hi(kk[3]), a);
             }
-            m[g] = mn;
+#pragma unroll
+            for (int off = 1; off < LPP; off <<= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+            sc[g] = a;
+          }
+        }
+        if (valid) {
+          const uint4 vw = *reinterpret_cast<const uint4*>(vb + (size_t)j * HD * 2 + cl * 16);
+          const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+          for (int g = 0; g < HW; ++g) {
+            if (g0 + g < G) {
+              const float mn = fmaxf(m[g], sc[g]);
+              const float cr = exp2_scale(m[g], mn), pe = exp2f(sc[g] - mn);
+              ls[g] = ls[g] * cr + pe;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                o[g][2 * q] = fmaf(o[g][2 * q], cr, pe * bf_lo(vv[q]));
+                o[g][2 * q + 1] = fmaf(o[g][2 * q + 1], cr, pe * bf_hi(vv[q]));
+              }
+              m[g] = mn;
+            }
           }
         }
       }
@@ -688,9 +893,9 @@ __device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it)
     if (lane == 0) mbar_arrive(&s.empty[slot]);
   }
 
-  // merge the sub-warps of this warp (lanes with the same chunk)
+  // merge the sub-warps of this warp (lanes with the same piece)
 #pragma unroll
-  for (int g = 0; g < kMaxGroup; ++g) {
+  for (int g = 0; g < HW; ++g) {
 #pragma unroll
     for (int off = LPP; off < 32; off <<= 1) {
       const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
@@ -706,47 +911,44 @@ __device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it)
       m[g] = M;
     }
   }
-  // merge the 16 warps: a 4-round tree through shared memory
+  // merge the warps of each head group: a tree through shared memory
   const int stride = HD + 2;
-  for (int k = kConsumerWarps / 2; k >= 1; k >>= 1) {
-    if (warp >= k && warp < 2 * k && sw == 0) {
-      float* ent = s.aux + (size_t)(warp - k) * kMaxGroup * stride;
+  float* aux = s.aux + (size_t)hg * (kConsumerWarps / 2) * HW * stride;
+  for (int k = WPH / 2; k >= 1; k >>= 1) {
+    if (in_group && wi >= k && wi < 2 * k && sw == 0) {
+      float* ent = aux + (size_t)(wi - k) * HW * stride;
 #pragma unroll
-      for (int g = 0; g < kMaxGroup; ++g) {
-        if (g < G) {
+      for (int g = 0; g < HW; ++g) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
-          if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
-        }
+        for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
+        if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
       }
     }
     bar_compute();
-    if (warp < k) {
-      const float* ent = s.aux + (size_t)warp * kMaxGroup * stride;
+    if (in_group && wi < k) {
+      const float* ent = aux + (size_t)wi * HW * stride;
 #pragma unroll
-      for (int g = 0; g < kMaxGroup; ++g) {
-        if (g < G) {
-          const float mo = ent[g * stride + HD], lo = ent[g * stride + HD + 1];
-          const float M = fmaxf(m[g], mo);
-          const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
-          ls[g] = ls[g] * fa + lo * fb;
+      for (int g = 0; g < HW; ++g) {
+        const float mo = ent[g * stride + HD], lo = ent[g * stride + HD + 1];
+        const float M = fmaxf(m[g], mo);
+        const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
+        ls[g] = ls[g] * fa + lo * fb;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[g][e] = o[g][e] * fa + ent[g * stride + cl * 8 + e] * fb;
-          m[g] = M;
-        }
+        for (int e = 0; e < 8; ++e) o[g][e] = o[g][e] * fa + ent[g * stride + cl * 8 + e] * fb;
+        m[g] = M;
       }
     }
     bar_compute();
   }
-  // this CTA's partial
-  if (warp == 0 && sw == 0) {
+  // this CTA's partial: warp 0 of each head group writes its heads
+  if (in_group && wi == 0 && sw == 0) {
     float* dst = p.attn_part + ((size_t)h * p.kv_chunks_max + c) * G * stride;
 #pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-      if (g < G) {
+    for (int g = 0; g < HW; ++g) {
+      if (g0 + g < G) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dst[g * stride + cl * 8 + e] = o[g][e];
-        if (cl == 0) { dst[g * stride + HD] = m[g]; dst[g * stride + HD + 1] = ls[g]; }
+        for (int e = 0; e < 8; ++e) dst[(g0 + g) * stride + cl * 8 + e] = o[g][e];
+        if (cl == 0) { dst[(g0 + g) * stride + HD] = m[g]; dst[(g0 + g) * stride + HD + 1] = ls[g]; }
       }
     }
   }
@@ -774,14 +976,13 @@ __device__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it)
 }
 
 // ------------------------------------------------------------------------------------------------
-// Grid argmax of the per-CTA LM maxima (lowest index on ties)
+// Grid argmax of the per-CTA LM maxima (lowest index on ties). Called by all compute threads.
 
-__device__ void grid_argmax(const Params& p, Smem& s) {
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x >= 32) return;
+__device__ __noinline__ void grid_argmax(const Params& p, Smem& s) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float bv = -CUDART_INF_F;
   int bi = 0x7fffffff;
-  for (int b = lane; b < p.grid; b += 32) {
+  for (int b = threadIdx.x; b < p.grid; b += kConsumerThreads) {
     const float v = __ldcg(p.am_val + b);
     const int i = __ldcg(p.am_idx + b);
     if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
@@ -792,7 +993,17 @@ __device__ void grid_argmax(const Params& p, Smem& s) {
     const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
     if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
   }
-  if (lane == 0) *p.next_token = (bi >= 0 && bi < p.V) ? bi : -1;
+  if (lane == 0) { s.misc->am_v[warp] = bv; s.misc->am_i[warp] = bi; }
+  bar_compute();
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float ov = s.misc->am_v[w];
+      const int oi = s.misc->am_i[w];
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    *p.next_token = (bi >= 0 && bi < p.V) ? bi : -1;
+  }
+  bar_compute();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -822,25 +1033,30 @@ __device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
   for (int ti = 0; ti < nt; ++ti) {
     const Task t = tasks[ti];
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_tasks_per_cta + ti) * 4 : nullptr;
-    if (tr && tid == 0) { tr[0] = ((unsigned long long)t.op << 32) | (unsigned long long)t.layer << 16 | (unsigned)ti; tr[1] = globaltimer(); }
+    if (tr && tid == 0) {
+      tr[0] = ((unsigned long long)t.op << 32) | (unsigned long long)t.layer << 16 | (unsigned)ti;
+      tr[1] = tr[2] = globaltimer();
+    }
     if (is_gemv(t.op)) {
       const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
       const bool w8 = i8 && !(t.op == OP_LM && p.tied);
       if (w8) {
         switch (g.gb) {
-          case 16: gemv_task<true, 16>(p, t, s, it, token); break;
-          case 8: gemv_task<true, 8>(p, t, s, it, token); break;
-          case 4: gemv_task<true, 4>(p, t, s, it, token); break;
-          default: gemv_task<true, 2>(p, t, s, it, token); break;
+          case 32: gemv_nr<true, 32>(p, t, s, it, token, tr, g.nr); break;
+          case 16: gemv_nr<true, 16>(p, t, s, it, token, tr, g.nr); break;
+          case 8: gemv_nr<true, 8>(p, t, s, it, token, tr, g.nr); break;
+          case 4: gemv_nr<true, 4>(p, t, s, it, token, tr, g.nr); break;
+          default: gemv_nr<true, 2>(p, t, s, it, token, tr, g.nr); break;
         }
       } else {
         switch (g.gb) {
-          case 16: gemv_task<false, 16>(p, t, s, it, token); break;
-          case 8: gemv_task<false, 8>(p, t, s, it, token); break;
-          default: gemv_task<false, 4>(p, t, s, it, token); break;
+          case 64: gemv_nr<false, 64>(p, t, s, it, token, tr, g.nr); break;
+          case 32: gemv_nr<false, 32>(p, t, s, it, token, tr, g.nr); break;
+          case 16: gemv_nr<false, 16>(p, t, s, it, token, tr, g.nr); break;
+          case 8: gemv_nr<false, 8>(p, t, s, it, token, tr, g.nr); break;
+          default: gemv_nr<false, 4>(p, t, s, it, token, tr, g.nr); break;
         }
       }
-      if (tr && tid == 0) tr[2] = globaltimer();
       if (t.op == OP_LM) {
         if (t.flags & kLastOfStage) {
           if (tid == 0) { p.am_val[blockIdx.x] = s.misc->lm_v; p.am_idx[blockIdx.x] = s.misc->lm_i; }
@@ -864,9 +1080,8 @@ __device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
         signal_counter(p, t.sig_ctr);
       }
     } else if (t.op == OP_ATTN) {
-      if (p.hd == 64) attn_task<64>(p, t, s, it);
-      else attn_task<128>(p, t, s, it);
-      if (tr && tid == 0) tr[2] = globaltimer();
+      if (p.hd == 64) attn_task<64>(p, t, s, it, tr);
+      else attn_task<128>(p, t, s, it, tr);
     } else if (t.op == OP_MERGE) {
       merge_head(p, t.a, attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max));
     } else if (t.op == OP_ARGMAX) {

@@ -58,21 +58,29 @@ std::string fmt(const char* f, long a = 0, long b = 0, long c = 0) {
 }  // namespace
 
 bool make_geom(int K, int esize, GemvGeom* g) {
+  // Bytes per thread per row: larger groups amortise the per-slot reduction and bookkeeping over
+  // more weight bytes (weight 1.0 for 32 B), smaller ones fit rows that larger ones do not divide.
+  // Each candidate is scored by that efficiency times the fraction of compute warps it keeps busy.
   int rb = K * esize;
   if (K <= 0 || rb > kSlotBytes) return false;
   bool found = false;
   double best = -1.0;
-  for (int gb : {16, 8, 4, 2}) {
-    if (gb < esize * 2 && esize == 2) continue;           // bf16: at least 2 elements per group
+  const int gbs[] = {64, 32, 16, 8, 4, 2};
+  const double eff[] = {1.0, 1.0, 0.8, 0.65, 0.5, 0.4};
+  for (int i = 0; i < 6; ++i) {
+    const int gb = gbs[i];
+    if (esize == 2 && gb < 4) continue;                   // bf16: at least 2 elements per group
+    if (esize == 1 && gb > 32) continue;                  // int8: at most 32 bytes per thread per row
     if (rb % (gb * 32) != 0) continue;
     int W = rb / gb / 32;
     int nr = (W + kConsumerWarps - 1) / kConsumerWarps;
-    if (nr > (esize == 1 ? 32 : 64) / gb) continue;       // activation registers (K <= 16384)
+    if (nr > (esize == 1 ? 32 : 64) / gb) continue;       // <= 32 activations per thread
     int wpg = W < kConsumerWarps ? W : kConsumerWarps;
     int rp = nr == 1 ? kConsumerWarps / wpg : 1;
     double bal = nr == 1 ? double(rp * wpg) / kConsumerWarps : double(W) / (nr * kConsumerWarps);
-    if (bal > best + 1e-9) {
-      best = bal;
+    double score = bal * eff[i];
+    if (score > best + 1e-9) {
+      best = score;
       int rs = kSlotBytes / rb;
       if (rs > 64) rs = 64;
       if (rs > 1 && (rs & 1)) rs -= 1;
