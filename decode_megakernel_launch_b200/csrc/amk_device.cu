@@ -122,6 +122,9 @@ struct Smem {
   Misc* misc;
 };
 
+extern __shared__ __align__(128) uint8_t smem_raw[];
+__device__ __forceinline__ Smem smem_view();
+
 __device__ __forceinline__ Smem carve(uint8_t* base) {
   Smem s;
   s.ring = base;
@@ -134,6 +137,9 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
   s.misc = reinterpret_cast<Misc*>(m + 2 * kSlots * 8);
   return s;
 }
+// The shared-memory view of this CTA, rebuilt from the dynamic shared-memory base (cheap pointer
+// arithmetic), so routines take no Smem argument that would otherwise live in local memory.
+__device__ __forceinline__ Smem smem_view() { return carve(smem_raw); }
 
 // ------------------------------------------------------------------------------------------------
 // Failure handling and waits
@@ -312,7 +318,8 @@ __device__ void prefetch_side_data(const Params& p, const Task& t, int token) {
 
 // Producer lane: issues every item of the CTA's byte stream into the ring in order, gated only by
 // the ring's empty barriers (never by other CTAs).
-__device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt, Smem& s) {
+__device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt) {
+  Smem s = smem_view();
   const uint64_t pol = policy_evict_first();
   int token = p.token;
   if (token < 0) token = __ldcg(p.next_token);
@@ -344,7 +351,7 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
 // GEMV
 
 // Block-wide sum over the compute threads in a fixed order (deterministic).
-__device__ float block_sum(float v, Smem& s) {
+__device__ float block_sum(float v, const Smem& s) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -475,8 +482,9 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 // groups per thread (geometry nr <= NR). For RMSNorm inputs the thread works on x * g and the
 // 1/rms factor is applied per row in the epilogue, so the input loads need one L2 round trip.
 template <bool I8, int GB, int NR>
-__device__ __noinline__ void gemv_task(const Params& p, const Task& t, Smem& s, uint32_t& it, int token,
-                          unsigned long long* tr) {
+__device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32_t it, int token,
+                                          unsigned long long* tr) {
+  const Smem s = smem_view();
   constexpr int ES = I8 ? 1 : 2;                        // weight element bytes
   constexpr int PB = GB < 16 ? GB : 16;                 // bytes per piece
   constexpr int NP = GB / PB;                           // pieces per group
@@ -715,19 +723,20 @@ __device__ __noinline__ void gemv_task(const Params& p, const Task& t, Smem& s, 
     }
     bar_compute();
   }
+  return it;
 }
 
 // Picks the register footprint: one group per thread, or the most the bytes per thread allow
 // (<= 32 int8 / 32 bf16 activations per thread).
 template <bool I8, int GB>
-__device__ __forceinline__ void gemv_nr(const Params& p, const Task& t, Smem& s, uint32_t& it, int token,
-                                        unsigned long long* tr, int nr) {
+__device__ __forceinline__ uint32_t gemv_nr(const Params& p, const Task& t, uint32_t it, int token,
+                                            unsigned long long* tr, int nr) {
   constexpr int NRMAX = (I8 ? 32 : 64) / GB;
   if constexpr (NRMAX <= 1) {
-    gemv_task<I8, GB, 1>(p, t, s, it, token, tr);
+    return gemv_task<I8, GB, 1>(p, t, it, token, tr);
   } else {
-    if (nr <= 1) gemv_task<I8, GB, 1>(p, t, s, it, token, tr);
-    else gemv_task<I8, GB, NRMAX>(p, t, s, it, token, tr);
+    if (nr <= 1) return gemv_task<I8, GB, 1>(p, t, it, token, tr);
+    return gemv_task<I8, GB, NRMAX>(p, t, it, token, tr);
   }
 }
 
@@ -783,7 +792,8 @@ __device__ __noinline__ void merge_head(const Params& p, int h, int C) {
 constexpr int kHeadsPerWarp = 2;
 
 template <int HD>
-__device__ __noinline__ void attn_task(const Params& p, const Task& t, Smem& s, uint32_t& it, unsigned long long* tr) {
+__device__ __noinline__ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long long* tr) {
+  const Smem s = smem_view();
   constexpr int LPP = HD * 2 / 16;       // lanes per position (one 16-byte piece each)
   constexpr int PPW = 32 / LPP;          // positions per warp step
   constexpr int NPS = kSlotBytes / (4 * HD);
@@ -798,7 +808,7 @@ __device__ __noinline__ void attn_task(const Params& p, const Task& t, Smem& s, 
   const int h = t.a, c = t.b, l = t.layer;
   const int P = p.pos + 1;
   const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
-  if (c >= C) return;
+  if (c >= C) return it;
   int cb, ce;
   attn_chunk_range(P, C, c, &cb, &ce);
 
@@ -952,7 +962,7 @@ __device__ __noinline__ void attn_task(const Params& p, const Task& t, Smem& s, 
       }
     }
   }
-  if (!p.sync) return;
+  if (!p.sync) return it;
   // ticket: the last chunk of this head to finish merges all of them and signals
   bar_compute();
   uint32_t* ticket = p.attn_ticket + l * p.Hkv + h;
@@ -973,12 +983,14 @@ __device__ __noinline__ void attn_task(const Params& p, const Task& t, Smem& s, 
     }
   }
   bar_compute();
+  return it;
 }
 
 // ------------------------------------------------------------------------------------------------
 // Grid argmax of the per-CTA LM maxima (lowest index on ties). Called by all compute threads.
 
-__device__ __noinline__ void grid_argmax(const Params& p, Smem& s) {
+__device__ __noinline__ void grid_argmax(const Params& p) {
+  const Smem s = smem_view();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float bv = -CUDART_INF_F;
   int bi = 0x7fffffff;
@@ -1009,7 +1021,8 @@ __device__ __noinline__ void grid_argmax(const Params& p, Smem& s) {
 // ------------------------------------------------------------------------------------------------
 // Compute warps
 
-__device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
+__device__ void compute(const Params& p, const Task* tasks, int nt) {
+  const Smem s = smem_view();
   const int tid = threadIdx.x;
   if (tid == 0) {
     int tok = p.token;
@@ -1042,19 +1055,19 @@ __device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
       const bool w8 = i8 && !(t.op == OP_LM && p.tied);
       if (w8) {
         switch (g.gb) {
-          case 32: gemv_nr<true, 32>(p, t, s, it, token, tr, g.nr); break;
-          case 16: gemv_nr<true, 16>(p, t, s, it, token, tr, g.nr); break;
-          case 8: gemv_nr<true, 8>(p, t, s, it, token, tr, g.nr); break;
-          case 4: gemv_nr<true, 4>(p, t, s, it, token, tr, g.nr); break;
-          default: gemv_nr<true, 2>(p, t, s, it, token, tr, g.nr); break;
+          case 32: it = gemv_nr<true, 32>(p, t, it, token, tr, g.nr); break;
+          case 16: it = gemv_nr<true, 16>(p, t, it, token, tr, g.nr); break;
+          case 8: it = gemv_nr<true, 8>(p, t, it, token, tr, g.nr); break;
+          case 4: it = gemv_nr<true, 4>(p, t, it, token, tr, g.nr); break;
+          default: it = gemv_nr<true, 2>(p, t, it, token, tr, g.nr); break;
         }
       } else {
         switch (g.gb) {
-          case 64: gemv_nr<false, 64>(p, t, s, it, token, tr, g.nr); break;
-          case 32: gemv_nr<false, 32>(p, t, s, it, token, tr, g.nr); break;
-          case 16: gemv_nr<false, 16>(p, t, s, it, token, tr, g.nr); break;
-          case 8: gemv_nr<false, 8>(p, t, s, it, token, tr, g.nr); break;
-          default: gemv_nr<false, 4>(p, t, s, it, token, tr, g.nr); break;
+          case 64: it = gemv_nr<false, 64>(p, t, it, token, tr, g.nr); break;
+          case 32: it = gemv_nr<false, 32>(p, t, it, token, tr, g.nr); break;
+          case 16: it = gemv_nr<false, 16>(p, t, it, token, tr, g.nr); break;
+          case 8: it = gemv_nr<false, 8>(p, t, it, token, tr, g.nr); break;
+          default: it = gemv_nr<false, 4>(p, t, it, token, tr, g.nr); break;
         }
       }
       if (t.op == OP_LM) {
@@ -1070,7 +1083,7 @@ __device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
             bar_compute();
             if (s.misc->flag) {
               __threadfence();
-              grid_argmax(p, s);
+              grid_argmax(p);
               if (tid == 0) *p.am_ticket = 0u;
             }
           }
@@ -1080,19 +1093,18 @@ __device__ void compute(const Params& p, const Task* tasks, int nt, Smem& s) {
         signal_counter(p, t.sig_ctr);
       }
     } else if (t.op == OP_ATTN) {
-      if (p.hd == 64) attn_task<64>(p, t, s, it, tr);
-      else attn_task<128>(p, t, s, it, tr);
+      if (p.hd == 64) it = attn_task<64>(p, t, it, tr);
+      else it = attn_task<128>(p, t, it, tr);
     } else if (t.op == OP_MERGE) {
       merge_head(p, t.a, attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max));
     } else if (t.op == OP_ARGMAX) {
-      grid_argmax(p, s);
+      grid_argmax(p);
     }
     if (tr && tid == 0) tr[3] = globaltimer();
   }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem s = carve(smem_raw);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
@@ -1107,10 +1119,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const Task* tasks = p.tasks + p.task_off[b];
   const int nt = p.task_off[b + 1] - p.task_off[b];
   if (threadIdx.x >= kConsumerThreads) {
-    if (threadIdx.x == kConsumerThreads) producer(p, tasks, nt, s);
+    if (threadIdx.x == kConsumerThreads) producer(p, tasks, nt);
     return;
   }
-  compute(p, tasks, nt, s);
+  compute(p, tasks, nt);
 }
 
 // ------------------------------------------------------------------------------------------------
