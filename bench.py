@@ -183,7 +183,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
     start = cfg.prefill_len + cfg.prompt_len
     span = cfg.decode_steps
     t_setup = time.time()
-    model = DeviceModel(cfg)
+    model = DeviceModel(cfg, options=dict(kv_block=args.kv_block) if args.kv_block else None)
     if cfg.prompt_len:            # fill the prompt's KV once (positions 0..P-1)
         for i, t in enumerate(__import__("decode_megakernel_launch_b200.synth", fromlist=["x"]).prompt_ids(cfg)):
             model.step(t, i)
@@ -365,6 +365,7 @@ def main():
     ap.add_argument("--impl", default="amk", choices=["amk", "reference"])
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-block", type=int, default=0, help="amk_options.kv_block (minimum positions per attention chunk)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (smaller cases for profiler captures; not a bench line)")
     args = ap.parse_args()

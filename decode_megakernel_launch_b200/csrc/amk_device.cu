@@ -173,6 +173,7 @@ __device__ bool spin_counter(const Params& p, int ctr, uint32_t target) {
 }
 
 // All compute threads call this; thread 0 waits, then the compute barrier publishes it.
+// All compute threads call this; thread 0 waits, then the compute barrier publishes it.
 __device__ __forceinline__ void wait_counter(const Params& p, int ctr, uint32_t mult) {
   if (threadIdx.x == 0) spin_counter(p, ctr, p.epoch * mult);
   bar_compute();
@@ -236,6 +237,19 @@ struct ItemCursor {
   int end = 0;      // GEMV: rows; ATTN: chunk end position
 };
 
+// Item range of a task: GEMV rows [0, t.b), or the positions [begin, end) of an attention chunk
+// (empty when the chunk is inactive at this position); other tasks stream nothing.
+__device__ __forceinline__ void task_range(const Params& p, const Task& t, int& begin, int& end) {
+  begin = end = 0;
+  if (t.op == OP_ATTN) {
+    const int P = p.pos + 1;
+    const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
+    if (t.b < C) attn_chunk_range(P, C, t.b, &begin, &end);
+  } else if (is_gemv(t.op)) {
+    end = t.b;
+  }
+}
+
 // Advances `c` to the next item; returns false at the end of the list. (src0, n0) and (src1, n1)
 // are the item's byte ranges (n1 = 0 for GEMV items; n0 = n1 = 0 for an attention block that holds
 // only the current position, which is written this step and patched in shared memory).
@@ -245,19 +259,7 @@ __device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor
     const Task& t = tasks[c.ti];
     if (!c.started) {
       c.started = true;
-      if (t.op == OP_ATTN) {
-        const int P = p.pos + 1;
-        const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
-        int cb = 0, ce = 0;
-        if (t.b < C) attn_chunk_range(P, C, t.b, &cb, &ce);
-        c.sub = cb;
-        c.end = ce;
-      } else if (is_gemv(t.op)) {
-        c.sub = 0;
-        c.end = t.b;
-      } else {
-        c.sub = c.end = 0;
-      }
+      task_range(p, t, c.sub, c.end);
     }
     if (c.sub < c.end) {
       if (t.op == OP_ATTN) {
@@ -743,44 +745,46 @@ __device__ __forceinline__ uint32_t gemv_nr(const Params& p, const Task& t, uint
 // ------------------------------------------------------------------------------------------------
 // Attention (split-KV flash decoding)
 
-__device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : exp2f(m - M); }
+// 2^x with the hardware approximation (relative error ~2^-22; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : fast_exp2(m - M); }
 
-// Log-sum-exp merge of the C chunk partials of KV head h into attn_out. Chunks are read 16 at a time
-// with all their loads in flight, folded into a running (max, sum, output) per element.
+// Log-sum-exp merge of the C chunk partials of KV head h into attn_out, in two passes whose loads
+// are all in flight together: (1) every (head, chunk) max and sum, turned into per-chunk weights
+// exp2(m_c - M) / L in shared memory; (2) every output element sums its C chunk values with them.
 __device__ __noinline__ void merge_head(const Params& p, int h, int C) {
-  constexpr int B = 8;
+  const Smem s = smem_view();
   const int G = p.Hq / p.Hkv, hd = p.hd;
   const int stride = hd + 2;
+  const float* base = p.attn_part + (size_t)h * p.kv_chunks_max * G * stride;
+  float* wgt = s.aux;                       // [G][C] weights (aux is free after the attention tree)
+  for (int idx = threadIdx.x; idx < G * C; idx += kConsumerThreads) {
+    const int g = idx / C, c = idx % C;
+    wgt[idx] = __ldcg(base + ((size_t)c * G + g) * stride + hd);
+    wgt[G * C + idx] = __ldcg(base + ((size_t)c * G + g) * stride + hd + 1);
+  }
+  bar_compute();
+  for (int g = threadIdx.x; g < G; g += kConsumerThreads) {
+    float M = -CUDART_INF_F, L = 0.f;
+    for (int c = 0; c < C; ++c) M = fmaxf(M, wgt[g * C + c]);
+    for (int c = 0; c < C; ++c) L += wgt[G * C + g * C + c] * exp2_scale(wgt[g * C + c], M);
+    const float invL = 1.f / L;
+    for (int c = 0; c < C; ++c) wgt[g * C + c] = exp2_scale(wgt[g * C + c], M) * invL;
+  }
+  bar_compute();
+  const size_t cstride = (size_t)G * stride;
   for (int idx = threadIdx.x; idx < G * hd; idx += kConsumerThreads) {
     const int g = idx / hd, e = idx % hd;
-    const float* base = p.attn_part + ((size_t)h * p.kv_chunks_max * G + g) * stride;
-    const size_t cstride = (size_t)G * stride;
-    float M = -CUDART_INF_F, Ls = 0.f, O = 0.f;
-    for (int c0 = 0; c0 < C; c0 += B) {
-      float mm[B], ll[B], oo[B];
-#pragma unroll
-      for (int i = 0; i < B; ++i) {
-        const bool v = c0 + i < C;
-        const float* pc = base + (size_t)(c0 + i) * cstride;
-        mm[i] = v ? __ldcg(pc + hd) : -CUDART_INF_F;
-        ll[i] = v ? __ldcg(pc + hd + 1) : 0.f;
-        oo[i] = v ? __ldcg(pc + e) : 0.f;
-      }
-      float Mn = M;
-#pragma unroll
-      for (int i = 0; i < B; ++i) Mn = fmaxf(Mn, mm[i]);
-      const float f = exp2_scale(M, Mn);
-      Ls *= f;
-      O *= f;
-#pragma unroll
-      for (int i = 0; i < B; ++i) {
-        const float fi = exp2_scale(mm[i], Mn);
-        Ls = fmaf(ll[i], fi, Ls);
-        O = fmaf(oo[i], fi, O);
-      }
-      M = Mn;
-    }
-    p.attn_out[(h * G + g) * hd + e] = O / Ls;
+    const float* pe = base + (size_t)g * stride + e;
+    const float* w = wgt + g * C;
+    float acc = 0.f;
+#pragma unroll 16
+    for (int c = 0; c < C; ++c) acc = fmaf(__ldcg(pe + (size_t)c * cstride), w[c], acc);
+    p.attn_out[(h * G + g) * hd + e] = acc;
   }
 }
 
@@ -886,7 +890,7 @@ __device__ __noinline__ uint32_t attn_task(const Params& p, const Task t, uint32
           for (int g = 0; g < HW; ++g) {
             if (g0 + g < G) {
               const float mn = fmaxf(m[g], sc[g]);
-              const float cr = exp2_scale(m[g], mn), pe = exp2f(sc[g] - mn);
+              const float cr = exp2_scale(m[g], mn), pe = fast_exp2(sc[g] - mn);
               ls[g] = ls[g] * cr + pe;
 #pragma unroll
               for (int q = 0; q < 4; ++q) {

@@ -23,8 +23,8 @@ namespace amk {
 constexpr int kConsumerWarps   = 16;
 constexpr int kConsumerThreads = kConsumerWarps * 32;      // 512 compute threads
 constexpr int kThreads         = kConsumerThreads + 32;    // + 1 producer (bulk-copy) warp
-constexpr int kSlotBytes       = 32768;                    // one bulk-copy ring slot
-constexpr int kSlots           = 6;                        // ring depth (192 KB in flight per SM)
+constexpr int kSlotBytes       = 65536;                    // one bulk-copy ring slot
+constexpr int kSlots           = 3;                        // ring depth (192 KB in flight per SM)
 constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block
 constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV task (scale cache)
 constexpr int kMaxGroup        = 4;                        // Hq / Hkv supported
