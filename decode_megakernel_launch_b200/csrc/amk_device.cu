@@ -1,8 +1,9 @@
 // Device code of libamk (sm_100a): the persistent decode kernel, its routines, and the weight packer.
 //
 // One CTA per SM, 17 warps: warp 16 is the producer, whose elected lane streams every byte this CTA
-// will read (weight rows of its GEMV tasks, KV rows of its attention chunk) into a 6 x 32 KB
-// shared-memory ring with cp.async.bulk, completion tracked by one mbarrier per slot. The producer
+// will read (weight rows of its GEMV tasks, KV rows of its attention chunk) into a kSlots x kSlotBytes
+// shared-memory ring with cp.async.bulk, completion tracked by one mbarrier per slot; at most
+// kInflight copies are outstanding at once. The producer
 // never waits on other CTAs, so the next tasks' weights arrive while the compute warps wait on a
 // counter: this is the "prefetch the next layer's weights while the current layer computes" of
 // "AutoMegaKernel: A Statically-Checked Agent Harness for Self-Retargeting Megakernel Synthesis"
@@ -70,6 +71,12 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.volatile.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -159,14 +166,41 @@ __device__ bool spin_counter(const Params& p, int ctr, uint32_t target) {
   if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
   if (ld_volatile(p.abort_flag)) return false;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(20);
-    if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
-    if ((it & 15) == 0) {
+  if constexpr (kPollWindow > 1) {
+    // kPollWindow relaxed loads in flight, staggered by kPollGapNs: a count that lands is seen about
+    // one L2 round trip later instead of up to two; the acquire fence orders what follows after it
+    uint32_t v[kPollWindow];
+#pragma unroll
+    for (int k = 0; k < kPollWindow; ++k) {
+      v[k] = ld_relaxed(c);
+      __nanosleep(kPollGapNs);
+    }
+    for (;;) {
+#pragma unroll
+      for (int k = 0; k < kPollWindow; ++k) {
+        if ((int32_t)(v[k] - target) >= 0) {
+          fence_acq_rel_gpu();
+          return true;
+        }
+        v[k] = ld_relaxed(c);
+        __nanosleep(kPollGapNs);
+      }
       if (ld_volatile(p.abort_flag)) return false;
       if (globaltimer() - t0 > p.timeout_ns) {
         raise_abort(p, (1u << 16) | (uint32_t)ctr);
         return false;
+      }
+    }
+  } else {
+    for (uint32_t it = 1;; ++it) {
+      __nanosleep(20);
+      if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
+      if ((it & 15) == 0) {
+        if (ld_volatile(p.abort_flag)) return false;
+        if (globaltimer() - t0 > p.timeout_ns) {
+          raise_abort(p, (1u << 16) | (uint32_t)ctr);
+          return false;
+        }
       }
     }
   }
@@ -179,12 +213,11 @@ __device__ __forceinline__ void wait_counter(const Params& p, int ctr, uint32_t 
   bar_compute();
 }
 
+// The caller has passed a compute barrier after the task's last global store; thread 0's release
+// reduction then orders every store of the CTA before the count (release is cumulative over what
+// the barrier made visible to thread 0), pairing with the acquire load in spin_counter.
 __device__ __forceinline__ void signal_counter(const Params& p, int ctr) {
-  // caller has passed a compute barrier after the task's last global store
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(p.ctr + ctr, 1u);
-  }
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.ctr + ctr) : "memory");
 }
 
 // Bounded wait on a ring mbarrier phase. Its bound is 4x the counter bound, so a stalled counter is
@@ -326,8 +359,8 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
   int token = p.token;
   if (token < 0) token = __ldcg(p.next_token);
   if (token < 0 || token >= p.V) token = 0;
-  ItemCursor cur;
-  uint32_t it = 0;
+  ItemCursor cur, pfc;
+  uint32_t it = 0, pf_it = 0;
   int last_task = -1;
   const uint8_t *a0, *a1;
   uint32_t n0, n1;
@@ -337,7 +370,53 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
       prefetch_side_data(p, tasks[cur.ti], token);
     }
     const int slot = it % kSlots;
-    if (it >= (uint32_t)kSlots) wait_slot(p, &s.empty[slot], ((it / kSlots) - 1) & 1, (3u << 16) | slot);
+    if (kPfItems > 0 && pf_it <= it) {   // the L2 warm-up cursor restarts just past this item
+      pfc = cur;
+      pf_it = it + 1;
+    }
+    if (it >= (uint32_t)kSlots) {
+      const uint32_t par = ((it / kSlots) - 1) & 1;
+      if (kPfItems > 0 && !mbar_try_wait(&s.empty[slot], par)) {
+        // the slot's previous item has landed but is still held: once that lasts kStallNs the
+        // compute warps are waiting on a counter, so warm L2 with what follows, paced
+        const uint64_t t0 = globaltimer();
+        uint64_t last = 0;
+        bool cur_warm = pf_it > it + 1;   // already warmed as a look-ahead item of an earlier stall
+        while (!mbar_try_wait(&s.empty[slot], par)) {
+          const uint64_t now = globaltimer();
+          if (now - t0 > 4 * p.timeout_ns) {
+            raise_abort(p, (3u << 16) | slot);
+            break;
+          }
+          if (now - t0 > kStallNs && now - last > kPfGapNs && pf_it < it + kPfItems &&
+              mbar_try_wait(&s.full[slot], par)) {
+            const uint8_t *b0, *b1;
+            uint32_t m0, m1;
+            if (!cur_warm) {   // this item first: it is copied as soon as the slot frees
+              if (n0) prefetch_bulk_l2(a0, n0);
+              if (n1) prefetch_bulk_l2(a1, n1);
+              cur_warm = true;
+              last = now;
+            } else if (next_item(p, tasks, nt, pfc, b0, m0, b1, m1)) {
+              if (m0) prefetch_bulk_l2(b0, m0);
+              if (m1) prefetch_bulk_l2(b1, m1);
+              ++pf_it;
+              last = now;
+            } else {
+              pf_it = 0xffffffffu;
+            }
+          }
+        }
+      } else {
+        wait_slot(p, &s.empty[slot], par, (3u << 16) | slot);
+      }
+    }
+    if (kInflight < kSlots && it >= (uint32_t)kInflight) {
+      // item it - kInflight must have landed; its slot cannot have been refilled yet (that needs
+      // item it - kInflight + kSlots > it), so the parity names that item's phase alone
+      const uint32_t j = it - kInflight;
+      wait_slot(p, &s.full[j % kSlots], (j / kSlots) & 1, (5u << 16) | (j % kSlots));
+    }
     if (n0 + n1 > 0) {
       mbar_expect_tx(&s.full[slot], n0 + n1);
       bulk_g2s(s.ring + slot * kSlotBytes, a0, n0, &s.full[slot], pol);
@@ -353,19 +432,6 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
 // GEMV
 
 // Block-wide sum over the compute threads in a fixed order (deterministic).
-__device__ float block_sum(float v, const Smem& s) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (lane == 0) s.misc->red[warp] = v;
-  bar_compute();
-  float t = 0.f;
-#pragma unroll
-  for (int w = 0; w < kConsumerWarps; ++w) t += s.misc->red[w];
-  bar_compute();
-  return t;
-}
-
 // Sum of 4 per-lane values for 4 rows over the warp; lanes with (lane & 7) == 0 return row
 // (lane >> 3) & 3's total (transposed butterfly: 6 shuffles for 4 rows).
 __device__ __forceinline__ float reduce4_rows(float a0, float a1, float a2, float a3) {
@@ -438,16 +504,20 @@ __device__ __forceinline__ int dot_chunk_i8(int acc, const uint32_t* w, const ui
 }
 
 // Vector loads of N consecutive elements (N in {2, 4, 8, 16}) into fp32 registers.
+// Vector loads of N consecutive elements of a vector written earlier in this launch by other CTAs.
+// They may allocate in L1 (the row partitions of a CTA read the same elements, and L1 merges those
+// requests): every such read follows, in this CTA, an acquire on the counter of the stage that wrote
+// the vector plus a CTA barrier, so by the memory model it observes the released values.
 template <int N>
-__device__ __forceinline__ void ld_f32_cg(const float* p, float* o) {   // written by other CTAs: L2 only
+__device__ __forceinline__ void ld_f32_ca(const float* p, float* o) {
   if constexpr (N >= 4) {
 #pragma unroll
     for (int i = 0; i < N / 4; ++i) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + i);
+      const float4 v = __ldca(reinterpret_cast<const float4*>(p) + i);
       o[4 * i] = v.x; o[4 * i + 1] = v.y; o[4 * i + 2] = v.z; o[4 * i + 3] = v.w;
     }
   } else {
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(p));
+    const float2 v = __ldca(reinterpret_cast<const float2*>(p));
     o[0] = v.x; o[1] = v.y;
   }
 }
@@ -501,7 +571,8 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
   const bool active = rp < g.rp;
   const bool norm = op == OP_QKV || op == OP_GU || op == OP_LM;
 
-  // ---- static data first (scales), so its latency hides behind the wait ----
+  // ---- static data first, so its latency hides behind the wait: row scales into shared memory,
+  //      this thread's RMSNorm gains into registers, this position's RoPE row into aux ----
   const uint16_t* sc = I8 ? gemv_scales(p, op, l) : nullptr;
   if (I8 && sc)
     for (int i = tid; i < nrows; i += kConsumerThreads) s.scale[i] = bf2f(__ldg(sc + row0 + i));
@@ -512,30 +583,29 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
     col[j] = j * g.wpg + wg;
     ok[j] = active && j < g.nr && col[j] < g.wg_total;
   }
+  const uint16_t* gain =
+      op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : op == OP_LM ? p.final_norm : nullptr;
+  if (op == OP_QKV)
+    for (int i = tid; i < p.hd; i += kConsumerThreads) s.aux[i] = __ldg(p.rope + (size_t)p.pos * p.hd + i);
 
   if (p.sync && first && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
   if (tr && tid == 0) tr[2] = globaltimer();
 
-  // ---- inputs: the RMS pass (coalesced) and this thread's own elements, all loads in flight ----
+  // ---- inputs: this thread's own elements with their RMSNorm gains and, for O / down, the
+  //      residual of the task's rows (x is final here: its last writer precedes the awaited stage),
+  //      all in one batch of loads ----
+  // Row partition 0 covers every input element exactly once, so its threads' squares sum to the
+  // RMSNorm statistic; each warp leaves its share in misc->red and the epilogue (behind its own
+  // barrier) finishes the sum, so the prologue has a single dependent L2 round trip and no barrier.
+  static_assert(kMaxTaskRows <= 2 * kConsumerThreads, "two residual rows per thread");
+  const bool resid = op == OP_O || op == OP_DOWN;
+  float rv0 = 0.f, rv1 = 0.f;
+  if (resid && tid < nrows) rv0 = __ldca(p.x + row0 + tid);
+  if (resid && tid + kConsumerThreads < nrows) rv1 = __ldca(p.x + row0 + tid + kConsumerThreads);
   const bool from_embed = op == OP_QKV && l == 0;
   const float* src = op == OP_O ? p.attn_out : op == OP_DOWN ? p.act : p.x;
   const uint16_t* erow = p.embed + (size_t)token * p.d;
-  const uint16_t* gain =
-      op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : op == OP_LM ? p.final_norm : nullptr;
   float ss = 0.f;
-  if (norm) {
-    for (int e = tid * 4; e < p.d; e += kConsumerThreads * 4) {
-      float v[4];
-      if (from_embed) {
-        uint32_t w2[2];
-        ld_bf16_words<4>(erow + e, w2);
-        v[0] = bf_lo(w2[0]); v[1] = bf_hi(w2[0]); v[2] = bf_lo(w2[1]); v[3] = bf_hi(w2[1]);
-      } else {
-        ld_f32_cg<4>(src + e, v);
-      }
-      ss = fmaf(v[0], v[0], fmaf(v[1], v[1], fmaf(v[2], v[2], fmaf(v[3], v[3], ss))));
-    }
-  }
   float xv[NR * NP * PE];
 #pragma unroll
   for (int j = 0; j < NR; ++j) {
@@ -550,11 +620,13 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
 #pragma unroll
           for (int k = 0; k < PE / 2; ++k) { xp[2 * k] = bf_lo(ew[k]); xp[2 * k + 1] = bf_hi(ew[k]); }
         } else {
-          ld_f32_cg<PE>(src + e, xp);
+          ld_f32_ca<PE>(src + e, xp);
         }
         if (norm) {
           uint32_t gw[PE / 2];
           ld_bf16_words<PE>(gain + e, gw);
+#pragma unroll
+          for (int k = 0; k < PE; ++k) ss = fmaf(xp[k], xp[k], ss);
 #pragma unroll
           for (int k = 0; k < PE / 2; ++k) { xp[2 * k] *= bf_lo(gw[k]); xp[2 * k + 1] *= bf_hi(gw[k]); }
         }
@@ -564,8 +636,12 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
       }
     }
   }
-  float inv = 1.f;
-  if (norm) inv = rsqrtf(block_sum(ss, s) / (float)p.d + p.eps);
+  if (norm) {
+    if (rp != 0) ss = 0.f;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s.misc->red[warp] = ss;
+  }
 
   uint32_t ah[I8 ? NR * NP * PE / 2 : 1];
   float asc[I8 ? NR * NP : 1];   // per-piece scale: activation = int16 * asc
@@ -583,6 +659,11 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
         ah[c * PE / 2 + k] = ((uint32_t)lo & 0xffffu) | ((uint32_t)hi << 16);
       }
     }
+  }
+
+  if (resid) {   // read back by other threads in the epilogue, behind its barrier
+    if (tid < nrows) s.aux[tid] = rv0;
+    if (tid + kConsumerThreads < nrows) s.aux[tid + kConsumerThreads] = rv1;
   }
 
   // ---- rows, one ring slot at a time ----
@@ -651,6 +732,13 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
     const int done = r0 + srows;
     if (done - blk_base == blk_rows || done == nrows) {
       bar_compute();
+      float inv = 1.f;
+      if (norm) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) t += s.misc->red[w];
+        inv = rsqrtf(t / (float)p.d + p.eps);
+      }
       const int bs = blk_base, bn = done - blk_base;
       auto rowsum = [&](int rr) {
         float acc = 0.f;
@@ -668,7 +756,7 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
           } else {
             const int hd = p.hd, head = gr / hd, i = (gr % hd) >> 1;
             if (head < p.Hq + p.Hkv) {
-              const float c = p.rope[((size_t)p.pos * (hd / 2) + i) * 2], sn = p.rope[((size_t)p.pos * (hd / 2) + i) * 2 + 1];
+              const float c = s.aux[2 * i], sn = s.aux[2 * i + 1];
               const float o0 = v0 * c - v1 * sn, o1 = v1 * c + v0 * sn;
               if (head < p.Hq) {
                 p.q[head * hd + i] = o0;
@@ -693,7 +781,7 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
             if (p.logits) p.logits[gr] = val;
             if (val > lm_v || (val == lm_v && gr < lm_i)) { lm_v = val; lm_i = gr; }
           } else {
-            p.x[gr] = __ldcg(p.x + gr) + val;
+            p.x[gr] = s.aux[bs + rr] + val;
           }
         }
       }
@@ -753,38 +841,44 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 __device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : fast_exp2(m - M); }
 
-// Log-sum-exp merge of the C chunk partials of KV head h into attn_out, in two passes whose loads
-// are all in flight together: (1) every (head, chunk) max and sum, turned into per-chunk weights
-// exp2(m_c - M) / L in shared memory; (2) every output element sums its C chunk values with them.
+// Log-sum-exp merge of the C chunk partials (unnormalised o, running max m in log2 units, sum l) of
+// KV head h into attn_out. One thread per (query head, element); a warp holds 32 elements of one
+// query head. Per block of 32 chunks, lane k loads chunk k's (m, l) while every lane loads its own
+// element of all 32 chunks' o, all in one batch (one L2 round trip; a query head's chunks are HD + 2
+// floats apart, so one base address and immediate offsets serve every load); the block max and the
+// weighted sum of l are warp reductions and each chunk's weight reaches the other lanes by shuffle.
+// Blocks fold into running (M, L, acc) with the usual rescaling, so any C works.
+template <int HD>
 __device__ __noinline__ void merge_head(const Params& p, int h, int C) {
-  const Smem s = smem_view();
-  const int G = p.Hq / p.Hkv, hd = p.hd;
-  const int stride = hd + 2;
-  const float* base = p.attn_part + (size_t)h * p.kv_chunks_max * G * stride;
-  float* wgt = s.aux;                       // [G][C] weights (aux is free after the attention tree)
-  for (int idx = threadIdx.x; idx < G * C; idx += kConsumerThreads) {
-    const int g = idx / C, c = idx % C;
-    wgt[idx] = __ldcg(base + ((size_t)c * G + g) * stride + hd);
-    wgt[G * C + idx] = __ldcg(base + ((size_t)c * G + g) * stride + hd + 1);
-  }
-  bar_compute();
-  for (int g = threadIdx.x; g < G; g += kConsumerThreads) {
-    float M = -CUDART_INF_F, L = 0.f;
-    for (int c = 0; c < C; ++c) M = fmaxf(M, wgt[g * C + c]);
-    for (int c = 0; c < C; ++c) L += wgt[G * C + g * C + c] * exp2_scale(wgt[g * C + c], M);
-    const float invL = 1.f / L;
-    for (int c = 0; c < C; ++c) wgt[g * C + c] = exp2_scale(wgt[g * C + c], M) * invL;
-  }
-  bar_compute();
-  const size_t cstride = (size_t)G * stride;
-  for (int idx = threadIdx.x; idx < G * hd; idx += kConsumerThreads) {
-    const int g = idx / hd, e = idx % hd;
-    const float* pe = base + (size_t)g * stride + e;
-    const float* w = wgt + g * C;
-    float acc = 0.f;
-#pragma unroll 16
-    for (int c = 0; c < C; ++c) acc = fmaf(__ldcg(pe + (size_t)c * cstride), w[c], acc);
-    p.attn_out[(h * G + g) * hd + e] = acc;
+  constexpr int stride = HD + 2;
+  const int G = p.Hq / p.Hkv, lane = threadIdx.x & 31;
+  for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerThreads) {   // G * HD: whole warps
+    const int g = idx / HD, e = idx % HD;
+    const float* pg = p.attn_part + ((size_t)h * G + g) * p.kv_chunks_max * stride;
+    float M = -CUDART_INF_F, L = 0.f, acc = 0.f;
+    for (int c0 = 0; c0 < C; c0 += 32) {
+      const int nb = min(32, C - c0);
+      const float* pc = pg + (size_t)c0 * stride;
+      float2 ml = make_float2(-CUDART_INF_F, 0.f);
+      if (lane < nb) ml = __ldcg(reinterpret_cast<const float2*>(pc + lane * stride + HD));
+      float ov[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) ov[k] = k < nb ? __ldcg(pc + k * stride + e) : 0.f;
+      float Mb = fmaxf(M, ml.x);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, o));
+      const float w = exp2_scale(ml.x, Mb);
+      float lsum = ml.y * w;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+      const float r = exp2_scale(M, Mb);
+      L = fmaf(L, r, lsum);
+      acc *= r;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) acc = fmaf(ov[k], __shfl_sync(0xffffffffu, w, k), acc);
+      M = Mb;
+    }
+    p.attn_out[(h * G + g) * HD + e] = acc / L;
   }
 }
 
@@ -925,65 +1019,53 @@ __device__ __noinline__ uint32_t attn_task(const Params& p, const Task t, uint32
       m[g] = M;
     }
   }
-  // merge the warps of each head group: a tree through shared memory
-  const int stride = HD + 2;
-  float* aux = s.aux + (size_t)hg * (kConsumerWarps / 2) * HW * stride;
-  for (int k = WPH / 2; k >= 1; k >>= 1) {
-    if (in_group && wi >= k && wi < 2 * k && sw == 0) {
-      float* ent = aux + (size_t)(wi - k) * HW * stride;
-#pragma unroll
-      for (int g = 0; g < HW; ++g) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
-        if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
-      }
-    }
-    bar_compute();
-    if (in_group && wi < k) {
-      const float* ent = aux + (size_t)wi * HW * stride;
-#pragma unroll
-      for (int g = 0; g < HW; ++g) {
-        const float mo = ent[g * stride + HD], lo = ent[g * stride + HD + 1];
-        const float M = fmaxf(m[g], mo);
-        const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
-        ls[g] = ls[g] * fa + lo * fb;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[g][e] = o[g][e] * fa + ent[g * stride + cl * 8 + e] * fb;
-        m[g] = M;
-      }
-    }
-    bar_compute();
-  }
-  // this CTA's partial: warp 0 of each head group writes its heads
-  if (in_group && wi == 0 && sw == 0) {
-    float* dst = p.attn_part + ((size_t)h * p.kv_chunks_max + c) * G * stride;
+  // every warp's (m, l, o) of its heads into aux, one barrier, then one thread per (query head,
+  // element) folds the warps of its head group and writes this CTA's partial of that element
+  constexpr int stride = HD + 2;
+  if (in_group && sw == 0) {
+    float* ent = s.aux + ((size_t)hg * WPH + wi) * HW * stride;
 #pragma unroll
     for (int g = 0; g < HW; ++g) {
-      if (g0 + g < G) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dst[(g0 + g) * stride + cl * 8 + e] = o[g][e];
-        if (cl == 0) { dst[(g0 + g) * stride + HD] = m[g]; dst[(g0 + g) * stride + HD + 1] = ls[g]; }
-      }
+      for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
+      if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
     }
   }
+  bar_compute();
+  for (int idx = tid; idx < G * HD; idx += kConsumerThreads) {
+    const int g = idx / HD, e = idx % HD;
+    const float* ent = s.aux + (size_t)(g / HW) * WPH * HW * stride + (g % HW) * stride;
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < WPH; ++w) M = fmaxf(M, ent[w * HW * stride + HD]);
+    float L = 0.f, acc = 0.f;
+    for (int w = 0; w < WPH; ++w) {
+      const float* ew = ent + w * HW * stride;
+      const float wt = exp2_scale(ew[HD], M);
+      L = fmaf(ew[HD + 1], wt, L);
+      acc = fmaf(ew[e], wt, acc);
+    }
+    float* dg = p.attn_part + (((size_t)h * G + g) * p.kv_chunks_max + c) * stride;
+    dg[e] = acc;
+    if (e == 0) { dg[HD] = M; dg[HD + 1] = L; }
+  }
   if (!p.sync) return it;
-  // ticket: the last chunk of this head to finish merges all of them and signals
+  // ticket: the last chunk of this head to finish merges all of them and signals. The ticket is an
+  // acquire-release atomic: it publishes this CTA's partial (made visible to thread 0 by the
+  // barrier) and, for the last arrival, acquires every earlier chunk's.
   bar_compute();
   uint32_t* ticket = p.attn_ticket + l * p.Hkv + h;
   if (tid == 0) {
-    __threadfence();
-    const uint32_t old = atomicAdd(ticket, 1u);
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
     s.misc->flag = (old == (uint32_t)(C - 1));
   }
   bar_compute();
   if (s.misc->flag) {
-    __threadfence();
-    merge_head(p, h, C);
+    merge_head<HD>(p, h, C);
     bar_compute();
     if (tid == 0) {
       *ticket = 0u;
-      __threadfence();
-      atomicAdd(p.ctr + t.sig_ctr, 1u);
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.ctr + t.sig_ctr) : "memory");
     }
   }
   bar_compute();
@@ -1100,7 +1182,9 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
       if (p.hd == 64) it = attn_task<64>(p, t, it, tr);
       else it = attn_task<128>(p, t, it, tr);
     } else if (t.op == OP_MERGE) {
-      merge_head(p, t.a, attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max));
+      const int C = attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max);
+      if (p.hd == 64) merge_head<64>(p, t.a, C);
+      else merge_head<128>(p, t.a, C);
     } else if (t.op == OP_ARGMAX) {
       grid_argmax(p);
     }

@@ -23,8 +23,48 @@ namespace amk {
 constexpr int kConsumerWarps   = 16;
 constexpr int kConsumerThreads = kConsumerWarps * 32;      // 512 compute threads
 constexpr int kThreads         = kConsumerThreads + 32;    // + 1 producer (bulk-copy) warp
-constexpr int kSlotBytes       = 65536;                    // one bulk-copy ring slot
-constexpr int kSlots           = 3;                        // ring depth (192 KB in flight per SM)
+// Ring geometry (compile-time; -DAMK_SLOT_BYTES / -DAMK_SLOTS / -DAMK_INFLIGHT override it).
+// kInflight bounds the copies the producer keeps outstanding: every other global access of the SM
+// queues behind them, so fewer bytes in flight than the ring holds keeps those accesses short
+// while a stalled consumer still lets the ring fill to kSlots ahead.
+#ifndef AMK_SLOT_BYTES
+#define AMK_SLOT_BYTES 65536
+#endif
+#ifndef AMK_SLOTS
+#define AMK_SLOTS 3
+#endif
+#ifndef AMK_INFLIGHT
+#define AMK_INFLIGHT 2
+#endif
+constexpr int kSlotBytes       = AMK_SLOT_BYTES;           // one bulk-copy ring slot
+constexpr int kSlots           = AMK_SLOTS;                // ring depth
+constexpr int kInflight        = AMK_INFLIGHT;             // outstanding copies, <= kSlots
+// While the compute warps hold a landed slot longer than kStallNs (they wait on a counter), the
+// producer warms L2 with up to kPfItems upcoming ring items, one per kPfGapNs (about one SM's share
+// of HBM bandwidth), so HBM keeps streaming through the stage transition. kPfItems = 0 disables it.
+#ifndef AMK_PF_ITEMS
+#define AMK_PF_ITEMS 6
+#endif
+#ifndef AMK_PF_GAP_NS
+#define AMK_PF_GAP_NS 1200
+#endif
+#ifndef AMK_PF_STALL_NS
+#define AMK_PF_STALL_NS 400
+#endif
+// Counter waits keep this many polling loads in flight, one issued every kPollGapNs.
+#ifndef AMK_POLL_WINDOW
+#define AMK_POLL_WINDOW 1
+#endif
+#ifndef AMK_POLL_GAP_NS
+#define AMK_POLL_GAP_NS 200
+#endif
+constexpr int kPfItems = AMK_PF_ITEMS;
+constexpr unsigned kPfGapNs = AMK_PF_GAP_NS;
+constexpr unsigned kStallNs = AMK_PF_STALL_NS;
+constexpr int kPollWindow = AMK_POLL_WINDOW;
+constexpr unsigned kPollGapNs = AMK_POLL_GAP_NS;
+static_assert(kInflight >= 1 && kInflight <= kSlots, "ring in-flight bound");
+static_assert(kSlotBytes % 256 == 0 && kSlotBytes >= 32768, "ring slot holds a 32 KB weight row");
 constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block
 constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV task (scale cache)
 constexpr int kMaxGroup        = 4;                        // Hq / Hkv supported
@@ -34,6 +74,7 @@ constexpr int kPartBytes       = kConsumerWarps * kRowBlock * 4;
 constexpr int kScaleBytes      = kMaxTaskRows * 4;
 constexpr int kMiscBytes       = 512;
 constexpr int kSmemBytes       = kRingBytes + kPartBytes + kAuxBytes + kScaleBytes + kMiscBytes;
+static_assert(kAuxBytes >= kMaxTaskRows * 4 && kAuxBytes >= 128 * 4, "aux holds a GEMV task's residual rows or a RoPE row");
 
 // ---- tasks -----------------------------------------------------------------------------------
 enum Op : uint16_t {
@@ -120,7 +161,7 @@ struct Params {
   float* q;                    // roped queries [Hq*hd]
   float* attn_out;             // merged attention [Hq*hd]
   float* act;                  // SwiGLU output [ffn]
-  float* attn_part;            // [Hkv][kv_chunks_max][G][hd + 2]
+  float* attn_part;            // [Hkv][G][kv_chunks_max][hd + 2]: o, then m and l of each chunk
   float* am_val;               // per-CTA LM maxima [grid]
   int*   am_idx;
   uint32_t* ctr;               // [L * CTR_PER_LAYER]

@@ -110,7 +110,7 @@ int check_dims(const amk_dims& d, std::string* msg) {
   GemvGeom g;
   if (!make_geom(d.d_model, es, &g) || !make_geom(qd, es, &g) || !make_geom(d.ffn, es, &g) ||
       !make_geom(d.d_model, 2, &g))
-    return bad("a weight row does not fit a 32 KB ring slot");
+    return bad("a weight row does not fit a ring slot");
   return AMK_OK;
 }
 

@@ -165,7 +165,8 @@ int  amk_decode_step_unfused(amk_handle* h, int token_id, int pos, float* logits
 
 /* Sticky device status without synchronizing: AMK_OK or AMK_ERR_DEVICE_TIMEOUT (a wait expired in
  * an earlier launch). `detail` (may be NULL) receives the raw status word: bits 0..15 the counter
- * or slot index that expired, bits 16..23 the wait kind (1 counter, 2 full slot, 3 empty slot). */
+ * or slot index that expired, bits 16..23 the wait kind (1 counter, 2 full slot, 3 empty slot,
+ * 4 next-token id out of range at launch, 5 producer waiting for its own copy to land). */
 int  amk_status(const amk_handle* h, uint32_t* detail);
 
 /* Last CUDA error string seen by this library on this thread ("" if none). */
