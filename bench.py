@@ -308,16 +308,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(secs, 1)}
 
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            tj = json.load(open(tpath))
-            ent = tj.get(cfg.name)
-            if ent and ent.get("kernel_source_hash") == _kernel_hash():
-                traffic = ent["bytes_per_launch"]
-        except Exception:
-            traffic = None
+    traffic = _dram_traffic(cfg.name, avg_bytes)
 
     if rank == 0:
         srt = sorted(per)
@@ -347,6 +338,22 @@ def run_gpu(args, cfg, rank, world, local_rank):
         }
         print(json.dumps(line), flush=True)
     model.close()
+
+
+def _dram_traffic(workload, algorithmic_bytes):
+    """DRAM read+write bytes per launch from the committed ncu summary: its measured traffic /
+    algorithmic ratio times this launch's algorithmic bytes, or None when the summary was taken on
+    other kernel sources (or is missing)."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_dram_traffic.md")
+    try:
+        for line in open(path):
+            if line.startswith("traffic:"):
+                kv = dict(tok.split("=", 1) for tok in line.split()[1:])
+                if kv.get("workload") == workload and kv.get("kernel") == _kernel_hash():
+                    return float(kv["ratio"]) * algorithmic_bytes
+    except (OSError, ValueError, KeyError):
+        return None
+    return None
 
 
 def _kernel_hash():
