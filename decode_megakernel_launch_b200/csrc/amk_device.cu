@@ -561,7 +561,7 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
   constexpr int PB = GB < 16 ? GB : 16;                 // bytes per piece
   constexpr int NP = GB / PB;                           // pieces per group
   constexpr int PE = PB / ES;                           // elements per piece
-  constexpr int NB = GB >= 64 ? 1 : GB >= 32 ? 2 : 4;   // rows per register batch
+  constexpr int NB = GB >= 64 ? AMK_NB64 : GB >= 32 ? AMK_NB32 : 4;   // rows per register batch
   constexpr int WPP = PB >= 4 ? PB / 4 : 1;             // weight words per piece
   const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -887,7 +887,10 @@ __device__ __noinline__ void merge_head(const Params& p, int h, int C) {
 // small: 2 x (max, sum, 8 outputs) per lane). Inside a warp, LPP lanes hold one 16-byte piece of a
 // key/value row (8 elements) and PPW positions are processed per step; each sub-warp keeps an online
 // softmax, merged across sub-warps by shuffles and across the group's warps by a shared-memory tree.
-constexpr int kHeadsPerWarp = 2;
+#ifndef AMK_HEADS_PER_WARP
+#define AMK_HEADS_PER_WARP 2
+#endif
+constexpr int kHeadsPerWarp = AMK_HEADS_PER_WARP;
 
 template <int HD>
 __device__ __noinline__ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long long* tr) {
@@ -1019,26 +1022,50 @@ __device__ __noinline__ uint32_t attn_task(const Params& p, const Task t, uint32
       m[g] = M;
     }
   }
-  // every warp's (m, l, o) of its heads into aux, one barrier, then one thread per (query head,
-  // element) folds the warps of its head group and writes this CTA's partial of that element
+  // every warp's (m, l, o) of its heads into aux, then one thread per (query head, element) folds
+  // the entries of its head group and writes this CTA's partial of that element. When one entry per
+  // warp would not fit aux (4 heads per warp), the upper half of each group's warps first folds into
+  // the lower half through aux (one more barrier), leaving half as many entries.
   constexpr int stride = HD + 2;
-  if (in_group && sw == 0) {
-    float* ent = s.aux + ((size_t)hg * WPH + wi) * HW * stride;
+  constexpr bool two_level = kConsumerWarps * HW * stride * 4 > kAuxBytes;
+  static_assert((kConsumerWarps / 2) * HW * stride * 4 <= kAuxBytes, "attention fold entries fit aux");
+  const int nent = two_level ? WPH / 2 : WPH;   // entries per head group
+  auto put_entry = [&](int slot_idx) {
+    float* ent = s.aux + (size_t)slot_idx * HW * stride;
 #pragma unroll
     for (int g = 0; g < HW; ++g) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
       if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
     }
+  };
+  if (two_level) {
+    if (in_group && wi >= nent && sw == 0) put_entry(hg * nent + wi - nent);
+    bar_compute();
+    if (in_group && wi < nent) {
+      const float* ent = s.aux + (size_t)(hg * nent + wi) * HW * stride;
+#pragma unroll
+      for (int g = 0; g < HW; ++g) {
+        const float mo = ent[g * stride + HD], lo = ent[g * stride + HD + 1];
+        const float M = fmaxf(m[g], mo);
+        const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
+        ls[g] = ls[g] * fa + lo * fb;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[g][e] = o[g][e] * fa + ent[g * stride + cl * 8 + e] * fb;
+        m[g] = M;
+      }
+    }
+    bar_compute();
   }
+  if (in_group && wi < nent && sw == 0) put_entry(hg * nent + wi);
   bar_compute();
   for (int idx = tid; idx < G * HD; idx += kConsumerThreads) {
     const int g = idx / HD, e = idx % HD;
-    const float* ent = s.aux + (size_t)(g / HW) * WPH * HW * stride + (g % HW) * stride;
+    const float* ent = s.aux + (size_t)(g / HW) * nent * HW * stride + (g % HW) * stride;
     float M = -CUDART_INF_F;
-    for (int w = 0; w < WPH; ++w) M = fmaxf(M, ent[w * HW * stride + HD]);
+    for (int w = 0; w < nent; ++w) M = fmaxf(M, ent[w * HW * stride + HD]);
     float L = 0.f, acc = 0.f;
-    for (int w = 0; w < WPH; ++w) {
+    for (int w = 0; w < nent; ++w) {
       const float* ew = ent + w * HW * stride;
       const float wt = exp2_scale(ew[HD], M);
       L = fmaf(ew[HD + 1], wt, L);

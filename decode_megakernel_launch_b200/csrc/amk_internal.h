@@ -67,6 +67,14 @@ static_assert(kInflight >= 1 && kInflight <= kSlots, "ring in-flight bound");
 static_assert(kSlotBytes % 256 == 0 && kSlotBytes >= 32768, "ring slot holds a 32 KB weight row");
 constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block
 constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV task (scale cache)
+// Rows per register batch of the GEMV inner loop for 64- and 32-byte groups (the transposed
+// butterfly reduces 2 or 4 rows at once).
+#ifndef AMK_NB64
+#define AMK_NB64 1
+#endif
+#ifndef AMK_NB32
+#define AMK_NB32 4
+#endif
 constexpr int kMaxGroup        = 4;                        // Hq / Hkv supported
 constexpr int kAuxBytes        = 8 * kMaxGroup * (128 + 2) * 4;   // attention cross-warp tree
 constexpr int kRingBytes       = kSlots * kSlotBytes;
