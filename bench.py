@@ -309,6 +309,12 @@ def run_gpu(args, cfg, rank, world, local_rank):
                "seconds": round(secs, 1)}
 
     traffic = _dram_traffic(cfg.name, avg_bytes)
+    comparator = None
+    if world == 1 and not args.no_comparator:
+        try:
+            comparator = run_bf16_comparator(cfg, min(args.steps, 64), 3)
+        except Exception as e:  # context only, never the headline
+            comparator = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
 
     if rank == 0:
         srt = sorted(per)
@@ -334,10 +340,148 @@ def run_gpu(args, cfg, rank, world, local_rank):
                         "launches_per_step": 6 * cfg.n_layers + 2,
                         "graph_ms_per_step": graph_ms},
             "cpu_baseline": cpu,
+            "bf16_cublas_graph": comparator,
             "setup_s": round(setup_s, 1),
         }
         print(json.dumps(line), flush=True)
     model.close()
+
+
+# ------------------------------------------------------------------------------------------------
+# Comparator: the same decode step as plain torch bf16 ops (matmuls on cuBLAS), one CUDA graph.
+
+class TorchBf16Step:
+    """One batch-1 decode step written with torch bf16 tensors on the GPU, for comparison only: every
+    linear is an `F.linear` (a cuBLAS GEMV), attention is `scaled_dot_product_attention` over the
+    whole cache with a position mask, and the step is recorded once as a CUDA graph whose replays
+    read the token and position from device tensors and advance them (greedy feedback), so a replay
+    is one full decode step with no host work. It is not the product path and shares no code with it.
+
+    `w` holds bf16 CUDA tensors in source row order: embed [V, d]; per layer lists attn_norm, ffn_norm
+    [d], wqkv [(Hq + 2 Hkv) hd, d], wo [d, Hq hd], wgu [2 ffn, d] (gate rows then up rows),
+    wd [d, ffn]; final_norm [d]; lm_head [V, d]. KV caches are bf16 [L][Hkv, max_seq, hd].
+    """
+
+    def __init__(self, cfg, w, max_seq, start, span):
+        import torch
+        self.cfg, self.w, self.max_seq = cfg, w, max_seq
+        dev = w["embed"].device
+        hd, L = cfg.head_dim, cfg.n_layers
+        self.k = [torch.zeros(cfg.n_kv_heads, max_seq, hd, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+        self.v = [torch.zeros_like(t) for t in self.k]
+        inv = torch.pow(torch.tensor(float(cfg.rope_theta), dtype=torch.float64),
+                        -2.0 * torch.arange(hd // 2, dtype=torch.float64) / hd)
+        ang = torch.arange(max_seq, dtype=torch.float64)[:, None] * inv[None, :]
+        self.cos = ang.cos().float().to(dev)
+        self.sin = ang.sin().float().to(dev)
+        self.ar = torch.arange(max_seq, device=dev)
+        self.tok = torch.zeros(1, dtype=torch.long, device=dev)
+        self.pos = torch.zeros(1, dtype=torch.long, device=dev)
+        self.logits = torch.zeros(cfg.vocab, dtype=torch.float32, device=dev)
+        self.start, self.span = start, span
+        self.graph = None
+
+    def _rms(self, x, g):
+        import torch
+        return (x * torch.rsqrt(x.pow(2).mean(-1, keepdim=True) + self.cfg.rms_eps) * g.float()).to(torch.bfloat16)
+
+    def _rope(self, t, cos, sin):
+        import torch
+        a, b = t[..., : t.shape[-1] // 2], t[..., t.shape[-1] // 2:]
+        return torch.cat([a * cos - b * sin, b * cos + a * sin], dim=-1)
+
+    def _step(self, advance):
+        import torch
+        import torch.nn.functional as F
+        c, w = self.cfg, self.w
+        hq, hkv, hd = c.n_q_heads, c.n_kv_heads, c.head_dim
+        pos = self.pos
+        cos, sin = self.cos.index_select(0, pos), self.sin.index_select(0, pos)
+        bias = torch.where(self.ar <= pos, 0.0, float("-inf")).view(1, 1, 1, -1).to(torch.bfloat16)
+        x = w["embed"].index_select(0, self.tok).float()
+        for l in range(c.n_layers):
+            qkv = F.linear(self._rms(x, w["attn_norm"][l]), w["wqkv"][l]).float()
+            q = self._rope(qkv[:, : hq * hd].view(hq, hd), cos, sin)
+            k = self._rope(qkv[:, hq * hd: (hq + hkv) * hd].view(hkv, hd), cos, sin)
+            v = qkv[:, (hq + hkv) * hd:].view(hkv, hd)
+            self.k[l].index_copy_(1, pos, k.to(torch.bfloat16).unsqueeze(1))
+            self.v[l].index_copy_(1, pos, v.to(torch.bfloat16).unsqueeze(1))
+            o = F.scaled_dot_product_attention(q.to(torch.bfloat16).view(1, hq, 1, hd), self.k[l].unsqueeze(0),
+                                               self.v[l].unsqueeze(0), attn_mask=bias, enable_gqa=True)
+            x = x + F.linear(o.reshape(1, hq * hd), w["wo"][l]).float()
+            gu = F.linear(self._rms(x, w["ffn_norm"][l]), w["wgu"][l]).float()
+            a = F.silu(gu[:, : c.ffn]) * gu[:, c.ffn:]
+            x = x + F.linear(a.to(torch.bfloat16), w["wd"][l]).float()
+        self.logits.copy_(F.linear(self._rms(x, w["final_norm"]), w["lm_head"]).float()[0])
+        if advance:
+            self.tok.copy_(torch.argmax(self.logits).view(1))
+            self.pos.copy_(self.start + torch.remainder(pos + 1 - self.start, self.span))
+
+    def step_eager(self, token, pos):
+        self.tok.fill_(token)
+        self.pos.fill_(pos)
+        self._step(advance=False)
+        return self.logits
+
+    def capture(self, token, pos):
+        import torch
+        self.tok.fill_(token)
+        self.pos.fill_(pos)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self._step(advance=False)            # library and kernel selection before capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._step(advance=True)
+        torch.cuda.synchronize()
+
+
+def run_bf16_comparator(cfg, steps, warmup):
+    """Times TorchBf16Step on random bf16 weights of `cfg`'s shape (values do not change the time;
+    the step itself is checked against the oracle on a small model by the GPU tests)."""
+    import torch
+    dev = "cuda"
+    gen = torch.Generator(device=dev).manual_seed(1234)
+
+    def rnd(*shape, scale=0.02):
+        return (torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+    c, L = cfg, cfg.n_layers
+    qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim
+    w = {"embed": rnd(c.vocab, c.d_model, scale=1.0), "final_norm": 1 + rnd(c.d_model),
+         "attn_norm": [1 + rnd(c.d_model) for _ in range(L)], "ffn_norm": [1 + rnd(c.d_model) for _ in range(L)],
+         "wqkv": [rnd(qkv, c.d_model) for _ in range(L)], "wo": [rnd(c.d_model, c.n_q_heads * c.head_dim) for _ in range(L)],
+         "wgu": [rnd(2 * c.ffn, c.d_model) for _ in range(L)], "wd": [rnd(c.d_model, c.ffn) for _ in range(L)]}
+    w["lm_head"] = w["embed"] if c.tied else rnd(c.vocab, c.d_model)
+    start = c.prefill_len + c.prompt_len
+    span = c.decode_steps
+    m = TorchBf16Step(c, w, start + span, start, span)
+    for l in range(L):
+        m.k[l][:, :start] = torch.randn(c.n_kv_heads, start, c.head_dim, generator=gen, device=dev).to(torch.bfloat16)
+        m.v[l][:, :start] = torch.randn(c.n_kv_heads, start, c.head_dim, generator=gen, device=dev).to(torch.bfloat16)
+    m.capture(1, start)
+    for _ in range(warmup):
+        m.graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        m.graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    wbytes = sum(t.numel() * 2 for k in ("wqkv", "wo", "wgu", "wd") for t in w[k])
+    wbytes += (0 if c.tied else w["lm_head"].numel() * 2) + (c.vocab * c.d_model * 2 if c.tied else 0)
+    kv_bytes = 2 * L * c.n_kv_heads * (start + span) * c.head_dim * 2
+    out = {"what": "torch bf16 decode step (F.linear = cuBLAS GEMV, SDPA over the masked cache) replayed as one "
+                   "CUDA graph; random bf16 weights of the same shape", "ms_per_step": ms, "tokens_per_s": 1000.0 / ms,
+           "bytes_per_step": wbytes + kv_bytes, "achieved_gbs": (wbytes + kv_bytes) / (ms / 1000.0) / 1e9}
+    del m, w
+    torch.cuda.empty_cache()
+    return out
 
 
 def _dram_traffic(workload, algorithmic_bytes):
@@ -372,6 +516,7 @@ def main():
     ap.add_argument("--impl", default="amk", choices=["amk", "reference"])
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparator", action="store_true", help="skip the torch bf16 CUDA-graph comparator")
     ap.add_argument("--kv-block", type=int, default=0, help="amk_options.kv_block (minimum positions per attention chunk)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (smaller cases for profiler captures; not a bench line)")
