@@ -563,7 +563,9 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
   constexpr int PE = PB / ES;                           // elements per piece
   constexpr int NB = GB >= 64 ? AMK_NB64 : GB >= 32 ? AMK_NB32 : 4;   // rows per register batch
   constexpr int WPP = PB >= 4 ? PB / 4 : 1;             // weight words per piece
-  const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
+  // The geometry is copied to registers once: it is reached through a generic pointer, and each
+  // shared-memory store in the row loop would otherwise force the compiler to read it again.
+  const GemvGeom g = p.geom[gemv_slot_of(t.op)];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int op = t.op, l = t.layer, row0 = t.a, nrows = t.b;
   const bool first = t.flags & kFirstOfStage;
