@@ -553,9 +553,15 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 // weights with packed fp32 FMAs. GB: weight bytes per thread per row; NR: compile-time bound on
 // groups per thread (geometry nr <= NR). For RMSNorm inputs the thread works on x * g and the
 // 1/rms factor is applied per row in the epilogue, so the input loads need one L2 round trip.
+// The hot GEMV instance (int8, 32-byte groups, one group per thread) is inlined into the kernel's
+// task loop: a non-inlined call saves and restores registers through local memory, whose lines
+// rarely stay in L1 next to 226 KB of shared memory, at every task boundary.
+#ifndef AMK_INLINE_HOT
+#define AMK_INLINE_HOT 1
+#endif
 template <bool I8, int GB, int NR>
-__device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32_t it, int token,
-                                          unsigned long long* tr) {
+__device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uint32_t it, int token,
+                                             unsigned long long* tr) {
   const Smem s = smem_view();
   constexpr int ES = I8 ? 1 : 2;                        // weight element bytes
   constexpr int PB = GB < 16 ? GB : 16;                 // bytes per piece
@@ -818,6 +824,12 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
   return it;
 }
 
+template <bool I8, int GB, int NR>
+__device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32_t it, int token,
+                                          unsigned long long* tr) {
+  return gemv_body<I8, GB, NR>(p, t, it, token, tr);
+}
+
 // Picks the register footprint: one group per thread, or the most the bytes per thread allow
 // (<= 32 int8 / 32 bf16 activations per thread).
 template <bool I8, int GB>
@@ -894,8 +906,16 @@ __device__ __noinline__ void merge_head(const Params& p, int h, int C) {
 #endif
 constexpr int kHeadsPerWarp = AMK_HEADS_PER_WARP;
 
+#ifndef AMK_INLINE_ATTN
+#define AMK_INLINE_ATTN 0
+#endif
 template <int HD>
-__device__ __noinline__ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long long* tr) {
+#if AMK_INLINE_ATTN
+__device__ __forceinline__
+#else
+__device__ __noinline__
+#endif
+uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long long* tr) {
   const Smem s = smem_view();
   constexpr int LPP = HD * 2 / 16;       // lanes per position (one 16-byte piece each)
   constexpr int PPW = 32 / LPP;          // positions per warp step
@@ -1170,7 +1190,11 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
       const bool w8 = i8 && !(t.op == OP_LM && p.tied);
       if (w8) {
         switch (g.gb) {
-          case 32: it = gemv_nr<true, 32>(p, t, it, token, tr, g.nr); break;
+          case 32:
+#if AMK_INLINE_HOT
+            if (g.nr <= 1) { it = gemv_body<true, 32, 1>(p, t, it, token, tr); break; }
+#endif
+            it = gemv_nr<true, 32>(p, t, it, token, tr, g.nr); break;
           case 16: it = gemv_nr<true, 16>(p, t, it, token, tr, g.nr); break;
           case 8: it = gemv_nr<true, 8>(p, t, it, token, tr, g.nr); break;
           case 4: it = gemv_nr<true, 4>(p, t, it, token, tr, g.nr); break;
