@@ -118,6 +118,7 @@ struct Misc {
   int lm_i;
 };
 static_assert(sizeof(Misc) + 2 * kSlots * 8 <= kMiscBytes, "misc region");
+static_assert(sizeof(Task) * kTaskCache == kTaskCacheBytes, "task cache region");
 
 struct Smem {
   uint8_t* ring;
@@ -1255,10 +1256,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
-  __syncthreads();
+  // this CTA's task list into shared memory when it fits (read at every task boundary by the
+  // producer and the compute warps; a global read there is an L2 round trip on the critical path)
   const int b = blockIdx.x;
   const Task* tasks = p.tasks + p.task_off[b];
   const int nt = p.task_off[b + 1] - p.task_off[b];
+  if (p.sync && nt <= kTaskCache) {   // the op-per-kernel launches read one or two tasks each
+    Task* cache = reinterpret_cast<Task*>(smem_raw + kSmemBytes - kTaskCacheBytes);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(tasks);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(cache);
+    for (int i = threadIdx.x; i < nt * (int)(sizeof(Task) / 4); i += kThreads) dst[i] = __ldg(src + i);
+    tasks = cache;
+  }
+  __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
     if (threadIdx.x == kConsumerThreads) producer(p, tasks, nt);
     return;

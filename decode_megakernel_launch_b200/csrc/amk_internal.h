@@ -81,7 +81,10 @@ constexpr int kRingBytes       = kSlots * kSlotBytes;
 constexpr int kPartBytes       = kConsumerWarps * kRowBlock * 4;
 constexpr int kScaleBytes      = kMaxTaskRows * 4;
 constexpr int kMiscBytes       = 512;
-constexpr int kSmemBytes       = kRingBytes + kPartBytes + kAuxBytes + kScaleBytes + kMiscBytes;
+constexpr int kTaskCache       = 192;                      // task list copied to shared memory when it fits
+constexpr int kTaskCacheBytes  = kTaskCache * 32;
+constexpr int kSmemBytes       = kRingBytes + kPartBytes + kAuxBytes + kScaleBytes + kMiscBytes + kTaskCacheBytes;
+static_assert(kSmemBytes <= 227 * 1024, "dynamic shared memory of one CTA");
 static_assert(kAuxBytes >= kMaxTaskRows * 4 && kAuxBytes >= 128 * 4, "aux holds a GEMV task's residual rows or a RoPE row");
 
 // ---- tasks -----------------------------------------------------------------------------------
