@@ -269,6 +269,8 @@ struct ItemCursor {
   int sub = 0;      // GEMV: first row of the item; ATTN: first position of the item
   bool started = false;
   int end = 0;      // GEMV: rows; ATTN: chunk end position
+  const uint8_t* base = nullptr;   // GEMV: the task's first weight row, read once per task (the layer's
+  int rb = 0, rs = 0;              //   pointer is a dependent global load); row bytes, rows per slot
 };
 
 // Item range of a task: GEMV rows [0, t.b), or the positions [begin, end) of an attention chunk
@@ -294,6 +296,12 @@ __device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor
     if (!c.started) {
       c.started = true;
       task_range(p, t, c.sub, c.end);
+      if (is_gemv(t.op) && c.sub < c.end) {
+        const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
+        c.rb = g.rb;
+        c.rs = g.rs;
+        c.base = static_cast<const uint8_t*>(gemv_weights(p, t.op, t.layer)) + (size_t)t.a * g.rb;
+      }
     }
     if (c.sub < c.end) {
       if (t.op == OP_ATTN) {
@@ -306,10 +314,9 @@ __device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor
         n0 = n1 = (uint32_t)ntma * (uint32_t)p.hd * 2u;
         c.sub = be;
       } else {
-        const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
-        const int n = min(g.rs, c.end - c.sub);
-        src0 = static_cast<const uint8_t*>(gemv_weights(p, t.op, t.layer)) + (size_t)(t.a + c.sub) * g.rb;
-        n0 = (uint32_t)n * (uint32_t)g.rb;
+        const int n = min(c.rs, c.end - c.sub);
+        src0 = c.base + (size_t)c.sub * c.rb;
+        n0 = (uint32_t)n * (uint32_t)c.rb;
         src1 = nullptr;
         n1 = 0;
         c.sub += n;
