@@ -48,6 +48,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe of a phase (try_wait may suspend the thread for a system-defined time).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
@@ -390,14 +402,16 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
         const uint64_t t0 = globaltimer();
         uint64_t last = 0;
         bool cur_warm = pf_it > it + 1;   // already warmed as a look-ahead item of an earlier stall
-        while (!mbar_try_wait(&s.empty[slot], par)) {
+        // non-blocking probes: a suspended try_wait would hold the producer past the warm-up times
+        while (!mbar_test_wait(&s.empty[slot], par)) {
+          __nanosleep(100);
           const uint64_t now = globaltimer();
           if (now - t0 > 4 * p.timeout_ns) {
             raise_abort(p, (3u << 16) | slot);
             break;
           }
           if (now - t0 > kStallNs && now - last > kPfGapNs && pf_it < it + kPfItems &&
-              mbar_try_wait(&s.full[slot], par)) {
+              mbar_test_wait(&s.full[slot], par)) {
             const uint8_t *b0, *b1;
             uint32_t m0, m1;
             if (!cur_warm) {   // this item first: it is copied as soon as the slot frees
