@@ -40,16 +40,17 @@ constexpr int kSlotBytes       = AMK_SLOT_BYTES;           // one bulk-copy ring
 constexpr int kSlots           = AMK_SLOTS;                // ring depth
 constexpr int kInflight        = AMK_INFLIGHT;             // outstanding copies, <= kSlots
 // While the compute warps hold a landed slot longer than kStallNs (they wait on a counter), the
-// producer warms L2 with up to kPfItems upcoming ring items, one per kPfGapNs (about one SM's share
-// of HBM bandwidth), so HBM keeps streaming through the stage transition. kPfItems = 0 disables it.
+// producer warms L2 with up to kPfItems upcoming ring items, one per kPfGapNs (a little faster than
+// one SM's share of HBM bandwidth), so HBM keeps streaming through the stage transition; 10 items
+// of 64 KB on 148 SMs use at most 97 MB of the 126 MB L2. kPfItems = 0 disables it.
 #ifndef AMK_PF_ITEMS
-#define AMK_PF_ITEMS 6
+#define AMK_PF_ITEMS 10
 #endif
 #ifndef AMK_PF_GAP_NS
-#define AMK_PF_GAP_NS 1200
+#define AMK_PF_GAP_NS 800
 #endif
 #ifndef AMK_PF_STALL_NS
-#define AMK_PF_STALL_NS 400
+#define AMK_PF_STALL_NS 200
 #endif
 // Counter waits keep this many polling loads in flight, one issued every kPollGapNs.
 #ifndef AMK_POLL_WINDOW
