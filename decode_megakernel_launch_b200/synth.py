@@ -55,7 +55,7 @@ class ModelConfig:
     prefill_len: int = 0       # KV positions 0..prefill_len-1 filled with N(0,1) before decoding
     decode_steps: int = 0      # greedy decode steps after the prompt / prefill
     compare_steps: int = 0     # decode steps the oracle is compared on
-    weight_dtype: str = "int8"  # "int8" (W8A16) or "bf16"
+    weight_dtype: str = "int8"  # "int8" (W8A16), "int4" (W4A16) or "bf16"
 
     @property
     def max_seq(self) -> int:
@@ -85,6 +85,9 @@ PRESETS = {
     "llama1b_long32k": ModelConfig("llama1b_long32k", 4, 16, 2048, 32, 8, 64, 8192, 128256, True, 5e5,
                                    prefill_len=32768, decode_steps=64, compare_steps=4),
 }
+# W4A16 variants of the same shapes (int4 weight-only, per-row bf16 scales)
+for _n in ("tiny", "llama1b", "llama8b"):
+    PRESETS[_n + "_int4"] = PRESETS[_n].with_(name=_n + "_int4", weight_dtype="int4")
 
 
 def preset(name: str, **overrides) -> ModelConfig:

@@ -1,4 +1,4 @@
-"""CPU oracle for one batch-1 Llama-family decode step on W8A16 (or bf16) weights.
+"""CPU oracle for one batch-1 Llama-family decode step on W8A16 (or W4A16, or bf16) weights.
 
 TEST INFRASTRUCTURE ONLY. This module is the slow, plain reference that the CUDA path is checked
 against. Only the tests, the smoke check and the bench's CPU-baseline leg may import it; the product
@@ -24,6 +24,10 @@ Readings where the pages are silent (each is also listed in the design notes):
   * W8A16 quantiser: per output row, s = bf16_rne(max|w| / 127), q = clamp(rne(w / s), -127, 127);
     the scale is rounded before q is formed, so dequantisation q * s is exact in fp32. A row of
     zeros (or a scale that rounds to 0) gets s = 0, q = 0.
+  * W4A16 ("int4 (lossy, 2.42x reduced weight traffic) weight-only", technical summary, "Key
+    Contributions"): the same per-row symmetric scheme with 7 in place of 127, q in [-7, 7]. The
+    pages give no group size; per-row scales with the tied embedding left in bf16 reproduce the
+    quoted 2.42x traffic reduction over bf16 for the 1B-shaped model.
   * Everything is fp32 except the tensors that are stored in bf16: embedding, gains, scales,
     bf16 weights and the KV cache.
   * Attention is causal and includes the current position; scale 1/sqrt(hd); query head i reads
@@ -52,17 +56,18 @@ def bf16_round(x: torch.Tensor) -> torch.Tensor:
     return x.to(F32).to(torch.bfloat16).to(F32)
 
 
-def quantize_rows(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
-    """W8A16 per-output-row symmetric quantiser (abstract: "int8 (W8A16) megakernel").
+def quantize_rows(w: torch.Tensor, qmax: int = 127) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-output-row symmetric weight quantiser: W8A16 with qmax = 127 (abstract: "int8 (W8A16)
+    megakernel"), W4A16 with qmax = 7 (technical summary, "Key Contributions": int4 weight-only).
 
     Returns (q int8 [rows, cols], s fp32 [rows] holding bf16 values) with
-    s = bf16_rne(max|w_row| / 127) and q = clamp(round_half_even(w / s), -127, 127).
+    s = bf16_rne(max|w_row| / qmax) and q = clamp(round_half_even(w / s), -qmax, qmax).
     """
     w = w.to(F32)
     amax = w.abs().amax(dim=1)
-    s = bf16_round(amax / 127.0)
+    s = bf16_round(amax / float(qmax))
     safe = torch.where(s > 0, s, torch.ones_like(s))
-    q = torch.round(w / safe[:, None]).clamp_(-127, 127)
+    q = torch.round(w / safe[:, None]).clamp_(-qmax, qmax)
     q = torch.where((s > 0)[:, None], q, torch.zeros_like(q))
     return q.to(torch.int8), s
 
@@ -169,6 +174,7 @@ class OracleModel:
         self.final_norm = synth.norm_gain(cfg, None, "final_norm").to(F32)
         self.attn_norm = [synth.norm_gain(cfg, l, "attn_norm").to(F32) for l in range(cfg.n_layers)]
         self.ffn_norm = [synth.norm_gain(cfg, l, "ffn_norm").to(F32) for l in range(cfg.n_layers)]
+        self.qmax = 7 if cfg.weight_dtype == "int4" else 127
         n_params = cfg.n_layers * (cfg.qkv_rows + 3 * cfg.ffn + cfg.n_q_heads * cfg.head_dim) * cfg.d_model
         self.keep_dq = (n_params < 400_000_000) if keep_dequantized is None else keep_dequantized
         self._store: Dict[Tuple[Optional[int], str], tuple] = {}
@@ -183,7 +189,7 @@ class OracleModel:
             w = torch.zeros_like(w)
         if self.cfg.weight_dtype == "bf16":
             return ("w", bf16_round(w))
-        q, s = quantize_rows(w)
+        q, s = quantize_rows(w, self.qmax)
         if self.keep_dq:
             return ("w", dequantize(q, s))
         return ("qs", q, s)
@@ -196,9 +202,10 @@ class OracleModel:
         return ent[1] if ent[0] == "w" else dequantize(ent[1], ent[2])
 
     def quantized(self, layer: Optional[int], which: str) -> Tuple[torch.Tensor, torch.Tensor]:
-        """(q, s) of an int8 matrix, recomputed from the seeded weight."""
+        """(q, s) of a quantised matrix (int8 values; within [-7, 7] for W4A16), recomputed from
+        the seeded weight."""
         w = synth.linear(self.cfg, layer, which)
-        return quantize_rows(w)
+        return quantize_rows(w, self.qmax)
 
 
 class OracleKV:

@@ -42,12 +42,12 @@ def test_bf16_round_matches_bitwise_rne():
     assert got == want
 
 
-def _quantize_py(row):
+def _quantize_py(row, qmax=127):
     amax = max(abs(v) for v in row)
-    s = _bf16_rne_py(_f32(amax / 127.0))
+    s = _bf16_rne_py(_f32(amax / float(qmax)))
     if s == 0.0:
         return [0] * len(row), 0.0
-    q = [max(-127, min(127, round(_f32(v / s)))) for v in row]
+    q = [max(-qmax, min(qmax, round(_f32(v / s)))) for v in row]
     return q, s
 
 
@@ -62,6 +62,39 @@ def test_quantizer_brute_force():
         qr, sr = _quantize_py([_f32(v) for v in w[r].tolist()])
         assert q[r].tolist() == qr
         assert s[r].item() == sr
+
+
+def test_quantizer_int4_brute_force():
+    """W4A16 reading: the same per-row scheme with qmax = 7, against pure-Python rounding."""
+    g = torch.Generator().manual_seed(2)
+    w = torch.randn(9, 40, generator=g) * 0.02
+    w[2] = 0.0
+    w[6, 1] = -0.3
+    w[7] = torch.linspace(-0.7, 0.7, 40)        # ties of w/s at +-0.5 steps
+    q, s = O.quantize_rows(w, 7)
+    for r in range(w.shape[0]):
+        qr, sr = _quantize_py([_f32(v) for v in w[r].tolist()], 7)
+        assert q[r].tolist() == qr
+        assert s[r].item() == sr
+
+
+def test_quantizer_int4_bounds_and_exact_dequant():
+    w = synth.normal(6, "q4bounds", (64, 512), std=0.02)
+    q, s = O.quantize_rows(w, 7)
+    assert int(q.min()) >= -7 and int(q.max()) <= 7
+    assert set(q.abs().amax(dim=1).tolist()) <= {6, 7}
+    assert torch.equal(O.bf16_round(s), s)
+    deq = O.dequantize(q, s)
+    assert torch.equal(deq.double(), q.double() * s.double()[:, None])
+    err = (w - deq).abs()
+    unclamped = (w / s[:, None]).abs() <= 7
+    assert bool((err[unclamped] <= (s[:, None] / 2).expand_as(w)[unclamped] * (1 + 1e-6)).all())
+    # the oracle model uses this quantiser for int4 configs
+    cfg = synth.preset("tiny_int4")
+    m = O.OracleModel(cfg)
+    q2, s2 = m.quantized(0, "wo")
+    assert int(q2.abs().max()) <= 7
+    assert torch.equal(m.weight(0, "wo"), O.dequantize(q2, s2))
 
 
 def test_quantizer_bounds_and_exact_dequant():
