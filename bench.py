@@ -28,6 +28,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 decode tokens/s (W8A16) and achieved HBM GB/s vs B200 peak"
+DTYPE_TEXT = {"int8": "w8a16 (int8 weights, f16 activations, fp32 accumulate)",
+              "int4": "w4a16 (int4 weights, f16 activations, fp32 accumulate)",
+              "bf16": "bf16 weights, fp32 activations and accumulate"}
+
+
+def metric_for(cfg) -> str:
+    """The headline metric names the W8A16 workload; other weight dtypes say theirs instead."""
+    tag = {"int8": "W8A16", "int4": "W4A16", "bf16": "bf16 weights"}[cfg.weight_dtype]
+    return METRIC.replace("W8A16", tag)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -159,7 +168,7 @@ def run_reference(args, cfg, rank, world):
     t1 = statistics.median(timed)
     value = 1.0 / (t1 + (cfg.n_layers - 1) * t_layer)
     sample = smp.describe(args.steps) + "; per-layer cost calibrated over the warm-up steps"
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": metric_for(cfg), "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": _workload_name(cfg)},
@@ -319,10 +328,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
     if rank == 0:
         srt = sorted(per)
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "metric": metric_for(cfg), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "w8a16 (int8 weights, f16 activations, fp32 accumulate)"
-            if cfg.weight_dtype == "int8" else "bf16 weights, fp32 activations and accumulate",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_TEXT[cfg.weight_dtype],
             "data": "synthetic (seeded random-init weights of the named shape, N(0,1) KV prefill)",
             "config": {"workload": _workload_name(cfg), "grid": info.grid, "threads": info.threads,
                        "smem_bytes": info.smem_bytes, "l2": "weights+KV per step far exceed the 126 MB L2; no flush",

@@ -92,7 +92,9 @@ extern "C" {
 const char* amk_last_cuda_error(void) { return g_cuda_error.c_str(); }
 
 size_t amk_packed_bytes(int rows, int cols, int dst_dtype) {
-  if (rows < 0 || cols < 0 || (dst_dtype != AMK_W_INT8 && dst_dtype != AMK_W_BF16)) return 0;
+  if (rows < 0 || cols < 0 || (dst_dtype != AMK_W_INT8 && dst_dtype != AMK_W_BF16 && dst_dtype != AMK_W_INT4))
+    return 0;
+  if (dst_dtype == AMK_W_INT4) return (cols & 1) ? 0 : (size_t)rows * (size_t)cols / 2;
   return (size_t)rows * (size_t)cols * (dst_dtype == AMK_W_INT8 ? 1 : 2);
 }
 
@@ -109,8 +111,9 @@ int amk_pack_weight(int role, const amk_dims* dims, const void* src, int src_dty
                     void* packed_out, void* scales_out, void* stream) {
   if (!src || !packed_out || rows < 1 || cols < 1) return AMK_ERR_INVALID_ARG;
   if (src_dtype != AMK_SRC_F32 && src_dtype != AMK_SRC_BF16) return AMK_ERR_INVALID_ARG;
-  if (dst_dtype != AMK_W_INT8 && dst_dtype != AMK_W_BF16) return AMK_ERR_INVALID_ARG;
-  if (dst_dtype == AMK_W_INT8 && !scales_out) return AMK_ERR_INVALID_ARG;
+  if (dst_dtype != AMK_W_INT8 && dst_dtype != AMK_W_BF16 && dst_dtype != AMK_W_INT4) return AMK_ERR_INVALID_ARG;
+  if (dst_dtype != AMK_W_BF16 && !scales_out) return AMK_ERR_INVALID_ARG;
+  if (dst_dtype == AMK_W_INT4 && (cols & 1)) return AMK_ERR_INVALID_ARG;
   if (role < AMK_ROLE_PLAIN || role > AMK_ROLE_LM_HEAD) return AMK_ERR_INVALID_ARG;
   int hd = 1, ffn = 0;
   if (role != AMK_ROLE_PLAIN) {
@@ -137,14 +140,15 @@ uint64_t amk_step_bytes(const amk_dims* d, int pos) {
   if (!d || pos < 0) return 0;
   const uint64_t L = d->n_layers, dm = d->d_model, hd = d->head_dim, hq = d->n_q_heads, hkv = d->n_kv_heads,
                  ffn = d->ffn, V = d->vocab;
-  const uint64_t es = d->weight_dtype == AMK_W_INT8 ? 1 : 2;
-  const uint64_t sc = d->weight_dtype == AMK_W_INT8 ? 2 : 0;   // one bf16 scale per row
+  const int wd = d->weight_dtype;
+  auto wb = [wd](uint64_t elems) { return wd == AMK_W_INT4 ? elems / 2 : wd == AMK_W_BF16 ? elems * 2 : elems; };
+  const uint64_t sc = wd == AMK_W_BF16 ? 0 : 2;   // one bf16 scale per row of quantised weights
   const uint64_t qkv_rows = (hq + 2 * hkv) * hd;
-  uint64_t per_layer = qkv_rows * dm * es + qkv_rows * sc            // QKV
-                       + dm * hq * hd * es + dm * sc                 // O
-                       + 2 * ffn * dm * es + 2 * ffn * sc            // gate + up
-                       + dm * ffn * es + dm * sc;                    // down
-  uint64_t head = d->tied_head ? V * dm * 2 : V * dm * es + V * sc;
+  uint64_t per_layer = wb(qkv_rows * dm) + qkv_rows * sc             // QKV
+                       + wb(dm * hq * hd) + dm * sc                  // O
+                       + wb(2 * ffn * dm) + 2 * ffn * sc             // gate + up
+                       + wb(dm * ffn) + dm * sc;                     // down
+  uint64_t head = d->tied_head ? V * dm * 2 : wb(V * dm) + V * sc;
   uint64_t gains = (2 * L + 1) * dm * 2;
   uint64_t kv = 2ull * L * hkv * (uint64_t)(pos + 1) * hd * 2;
   return L * per_layer + head + dm * 2 /*embedding row*/ + gains + kv;
@@ -182,7 +186,7 @@ int amk_create(const amk_dims* dims, const amk_weights* w, const amk_options* op
     return rc;
   }
   const int L = d.n_layers;
-  const bool i8 = d.weight_dtype == AMK_W_INT8;
+  const bool i8 = d.weight_dtype != AMK_W_BF16;   // quantised (int8 or int4) weights carry row scales
   // pointer checks
   if (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->k_cache) || !aligned16(w->v_cache) ||
       !w->attn_norm || !w->ffn_norm || !w->wqkv || !w->wo || !w->wgu || !w->wdown)

@@ -355,7 +355,7 @@ __device__ __forceinline__ void prefetch_bulk_l2(const void* a, uint32_t bytes) 
 __device__ void prefetch_side_data(const Params& p, const Task& t, int token) {
   if (!is_gemv(t.op)) return;
   const uint16_t* sc = gemv_scales(p, t.op, t.layer);
-  if (p.wdtype == AMK_W_INT8 && sc && t.b > 0) {
+  if (p.wdtype != AMK_W_BF16 && sc && t.b > 0) {
     const char* b = reinterpret_cast<const char*>(sc + t.a);
     const int bytes = t.b * 2;
     for (int o = 0; o < bytes; o += 128) prefetch_line_l2(b + o);
@@ -571,9 +571,9 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 }
 
 // One GEMV task: rows [t.a, t.a + t.b) of the op's packed matrix against this step's input vector.
-// I8: int8 weights, dp2a against int16 activations quantised per 16-byte piece; otherwise bf16
-// weights with packed fp32 FMAs. GB: weight bytes per thread per row; NR: compile-time bound on
-// groups per thread (geometry nr <= NR). For RMSNorm inputs the thread works on x * g and the
+// WK (weight kind): 1 int8 and 2 int4 weights, dp2a against int16 activations quantised per
+// 16-byte piece; 0 bf16 weights with packed fp32 FMAs. GB: weight bytes per thread per row; NR:
+// compile-time bound on groups per thread (geometry nr <= NR). For RMSNorm inputs the thread works on x * g and the
 // 1/rms factor is applied per row in the epilogue, so the input loads need one L2 round trip.
 // The hot GEMV instance (int8, 32-byte groups, one group per thread) is inlined into the kernel's
 // task loop: a non-inlined call saves and restores registers through local memory, whose lines
@@ -581,14 +581,17 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 #ifndef AMK_INLINE_HOT
 #define AMK_INLINE_HOT 1
 #endif
-template <bool I8, int GB, int NR>
+template <int WK>
+__device__ __forceinline__ int elem_of_byte(int b) { return WK == 0 ? b / 2 : WK == 1 ? b : b * 2; }
+
+template <int WK, int GB, int NR>
 __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uint32_t it, int token,
                                              unsigned long long* tr) {
   const Smem s = smem_view();
-  constexpr int ES = I8 ? 1 : 2;                        // weight element bytes
+  constexpr bool IQ = WK != 0;                          // quantised weights: row scales, dp2a
   constexpr int PB = GB < 16 ? GB : 16;                 // bytes per piece
   constexpr int NP = GB / PB;                           // pieces per group
-  constexpr int PE = PB / ES;                           // elements per piece
+  constexpr int PE = WK == 0 ? PB / 2 : WK == 1 ? PB : PB * 2;   // elements per piece
   constexpr int NB = GB >= 64 ? AMK_NB64 : GB >= 32 ? AMK_NB32 : 4;   // rows per register batch
   constexpr int WPP = PB >= 4 ? PB / 4 : 1;             // weight words per piece
   // The geometry is copied to registers once: it is reached through a generic pointer, and each
@@ -603,8 +606,8 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
 
   // ---- static data first, so its latency hides behind the wait: row scales into shared memory,
   //      this thread's RMSNorm gains into registers, this position's RoPE row into aux ----
-  const uint16_t* sc = I8 ? gemv_scales(p, op, l) : nullptr;
-  if (I8 && sc)
+  const uint16_t* sc = IQ ? gemv_scales(p, op, l) : nullptr;
+  if (IQ && sc)
     for (int i = tid; i < nrows; i += kConsumerThreads) s.scale[i] = bf2f(__ldg(sc + row0 + i));
   bool ok[NR];
   int col[NR];
@@ -642,7 +645,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
 #pragma unroll
     for (int c = 0; c < NP; ++c) {
       float* xp = &xv[(j * NP + c) * PE];
-      const int e = piece_offset<GB>(col[j], lane, c) / ES;
+      const int e = elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c));
       if (ok[j]) {
         if (from_embed) {
           uint32_t ew[PE / 2];
@@ -673,9 +676,10 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
     if (lane == 0) s.misc->red[warp] = ss;
   }
 
-  uint32_t ah[I8 ? NR * NP * PE / 2 : 1];
-  float asc[I8 ? NR * NP : 1];   // per-piece scale: activation = int16 * asc
-  if constexpr (I8) {
+  uint32_t ah[IQ ? NR * NP * PE / 2 : 1];
+  float asc[IQ ? NR * NP : 1];   // per-piece scale: activation = int16 * asc
+  int sa[WK == 2 ? NR * NP : 1];  // int4: per-piece sum of the int16 activations (nibble offset 8)
+  if constexpr (IQ) {
 #pragma unroll
     for (int c = 0; c < NR * NP; ++c) {
       float amax = 0.f;
@@ -683,10 +687,26 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
       for (int k = 0; k < PE; ++k) amax = fmaxf(amax, fabsf(xv[c * PE + k]));
       const float q = amax > 0.f ? 32767.f / amax : 0.f;
       asc[c] = amax * (1.f / 32767.f);
+      auto qa = [&](int k) { return __float2int_rn(xv[c * PE + k] * q); };
+      auto pack2 = [](int lo, int hi) { return ((uint32_t)lo & 0xffffu) | ((uint32_t)hi << 16); };
+      if constexpr (WK == 1) {
 #pragma unroll
-      for (int k = 0; k < PE / 2; ++k) {
-        const int lo = __float2int_rn(xv[c * PE + 2 * k] * q), hi = __float2int_rn(xv[c * PE + 2 * k + 1] * q);
-        ah[c * PE / 2 + k] = ((uint32_t)lo & 0xffffu) | ((uint32_t)hi << 16);
+        for (int k = 0; k < PE / 2; ++k) ah[c * PE / 2 + k] = pack2(qa(2 * k), qa(2 * k + 1));
+      } else {
+        // a weight word holds elements 8m..8m+7 as nibbles: its low nibbles (elements 0, 2, 4, 6)
+        // and high nibbles (1, 3, 5, 7) meet activation words (x0, x2), (x4, x6), (x1, x3), (x5, x7)
+        int sum = 0;
+#pragma unroll
+        for (int m = 0; m < PE / 8; ++m) {
+          const int x0 = qa(8 * m), x1 = qa(8 * m + 1), x2 = qa(8 * m + 2), x3 = qa(8 * m + 3);
+          const int x4 = qa(8 * m + 4), x5 = qa(8 * m + 5), x6 = qa(8 * m + 6), x7 = qa(8 * m + 7);
+          ah[c * PE / 2 + 4 * m + 0] = pack2(x0, x2);
+          ah[c * PE / 2 + 4 * m + 1] = pack2(x4, x6);
+          ah[c * PE / 2 + 4 * m + 2] = pack2(x1, x3);
+          ah[c * PE / 2 + 4 * m + 3] = pack2(x5, x7);
+          sum += x0 + x1 + x2 + x3 + x4 + x5 + x6 + x7;
+        }
+        sa[c] = sum;
       }
     }
   }
@@ -723,8 +743,22 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
                 for (int c = 0; c < NP; ++c) {
                   uint32_t w[WPP];
                   lds_group<PB>(rowp + piece_offset<GB>(col[j], lane, c), w);
-                  if constexpr (I8) {
+                  if constexpr (WK == 1) {
                     const int acc = dot_chunk_i8<PE>(0, w, &ah[(j * NP + c) * PE / 2]);
+                    v = fmaf((float)acc, asc[j * NP + c], v);
+                  } else if constexpr (WK == 2) {
+                    // nibbles stored as q + 8: dot(a, u) - 8 * sum(a) = dot(a, q), exact in int32
+                    const uint32_t* a4 = &ah[(j * NP + c) * PE / 2];
+                    int acc = 0;
+#pragma unroll
+                    for (int k = 0; k < WPP; ++k) {
+                      const uint32_t lo = w[k] & 0x0f0f0f0fu, hi = (w[k] >> 4) & 0x0f0f0f0fu;
+                      acc = __dp2a_lo((int)a4[4 * k + 0], (int)lo, acc);
+                      acc = __dp2a_hi((int)a4[4 * k + 1], (int)lo, acc);
+                      acc = __dp2a_lo((int)a4[4 * k + 2], (int)hi, acc);
+                      acc = __dp2a_hi((int)a4[4 * k + 3], (int)hi, acc);
+                    }
+                    acc -= 8 * sa[j * NP + c];
                     v = fmaf((float)acc, asc[j * NP + c], v);
                   } else {
                     unsigned long long acc2 = 0ull;
@@ -774,7 +808,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
         float acc = 0.f;
         for (int w = 0; w < g.wpg; ++w) acc += s.part[w * kRowBlock + rr];
         acc *= inv;
-        return I8 && sc ? acc * s.scale[bs + rr] : acc;
+        return IQ && sc ? acc * s.scale[bs + rr] : acc;
       };
       if (op == OP_QKV || op == OP_GU) {
         for (int pr = tid; pr < bn / 2; pr += kConsumerThreads) {
@@ -846,23 +880,23 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
   return it;
 }
 
-template <bool I8, int GB, int NR>
+template <int WK, int GB, int NR>
 __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32_t it, int token,
                                           unsigned long long* tr) {
-  return gemv_body<I8, GB, NR>(p, t, it, token, tr);
+  return gemv_body<WK, GB, NR>(p, t, it, token, tr);
 }
 
 // Picks the register footprint: one group per thread, or the most the bytes per thread allow
 // (<= 32 int8 / 32 bf16 activations per thread).
-template <bool I8, int GB>
+template <int WK, int GB>
 __device__ __forceinline__ uint32_t gemv_nr(const Params& p, const Task& t, uint32_t it, int token,
                                             unsigned long long* tr, int nr) {
-  constexpr int NRMAX = (I8 ? 32 : 64) / GB;
+  constexpr int NRMAX = (WK == 0 ? 64 : WK == 1 ? 32 : 16) / GB;
   if constexpr (NRMAX <= 1) {
-    return gemv_task<I8, GB, 1>(p, t, it, token, tr);
+    return gemv_task<WK, GB, 1>(p, t, it, token, tr);
   } else {
-    if (nr <= 1) return gemv_task<I8, GB, 1>(p, t, it, token, tr);
-    return gemv_task<I8, GB, NRMAX>(p, t, it, token, tr);
+    if (nr <= 1) return gemv_task<WK, GB, 1>(p, t, it, token, tr);
+    return gemv_task<WK, GB, NRMAX>(p, t, it, token, tr);
   }
 }
 
@@ -1199,7 +1233,6 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
     for (int r = tid; r < n; r += kConsumerThreads) p.x[r0 + r] = bf2f(p.embed[(size_t)token * p.d + r0 + r]);
   }
   uint32_t it = 0;
-  const bool i8 = p.wdtype == AMK_W_INT8;
   for (int ti = 0; ti < nt; ++ti) {
     const Task t = tasks[ti];
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_tasks_per_cta + ti) * 4 : nullptr;
@@ -1209,26 +1242,32 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
     }
     if (is_gemv(t.op)) {
       const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
-      const bool w8 = i8 && !(t.op == OP_LM && p.tied);
-      if (w8) {
+      const int wk = t.op == OP_LM && p.tied ? AMK_W_BF16 : p.wdtype;   // a tied head reads the bf16 table
+      if (wk == AMK_W_INT8) {
         switch (g.gb) {
           case 32:
 #if AMK_INLINE_HOT
-            if (g.nr <= 1) { it = gemv_body<true, 32, 1>(p, t, it, token, tr); break; }
+            if (g.nr <= 1) { it = gemv_body<1, 32, 1>(p, t, it, token, tr); break; }
 #endif
-            it = gemv_nr<true, 32>(p, t, it, token, tr, g.nr); break;
-          case 16: it = gemv_nr<true, 16>(p, t, it, token, tr, g.nr); break;
-          case 8: it = gemv_nr<true, 8>(p, t, it, token, tr, g.nr); break;
-          case 4: it = gemv_nr<true, 4>(p, t, it, token, tr, g.nr); break;
-          default: it = gemv_nr<true, 2>(p, t, it, token, tr, g.nr); break;
+            it = gemv_nr<1, 32>(p, t, it, token, tr, g.nr); break;
+          case 16: it = gemv_nr<1, 16>(p, t, it, token, tr, g.nr); break;
+          case 8: it = gemv_nr<1, 8>(p, t, it, token, tr, g.nr); break;
+          case 4: it = gemv_nr<1, 4>(p, t, it, token, tr, g.nr); break;
+          default: it = gemv_nr<1, 2>(p, t, it, token, tr, g.nr); break;
+        }
+      } else if (wk == AMK_W_INT4) {
+        switch (g.gb) {
+          case 16: it = gemv_nr<2, 16>(p, t, it, token, tr, g.nr); break;
+          case 8: it = gemv_nr<2, 8>(p, t, it, token, tr, g.nr); break;
+          default: it = gemv_nr<2, 4>(p, t, it, token, tr, g.nr); break;
         }
       } else {
         switch (g.gb) {
-          case 64: it = gemv_nr<false, 64>(p, t, it, token, tr, g.nr); break;
-          case 32: it = gemv_nr<false, 32>(p, t, it, token, tr, g.nr); break;
-          case 16: it = gemv_nr<false, 16>(p, t, it, token, tr, g.nr); break;
-          case 8: it = gemv_nr<false, 8>(p, t, it, token, tr, g.nr); break;
-          default: it = gemv_nr<false, 4>(p, t, it, token, tr, g.nr); break;
+          case 64: it = gemv_nr<0, 64>(p, t, it, token, tr, g.nr); break;
+          case 32: it = gemv_nr<0, 32>(p, t, it, token, tr, g.nr); break;
+          case 16: it = gemv_nr<0, 16>(p, t, it, token, tr, g.nr); break;
+          case 8: it = gemv_nr<0, 8>(p, t, it, token, tr, g.nr); break;
+          default: it = gemv_nr<0, 4>(p, t, it, token, tr, g.nr); break;
         }
       }
       if (t.op == OP_LM) {
@@ -1325,15 +1364,23 @@ __global__ void pack_kernel(int role, int hd, int ffn, const void* src, int src_
     if (threadIdx.x == 0) red[0] = a;
   }
   __syncthreads();
-  const uint16_t sb = f2bf(__fdiv_rn(red[0], 127.f));
+  const float qmax = dst_dtype == AMK_W_INT4 ? 7.f : 127.f;
+  const uint16_t sb = f2bf(__fdiv_rn(red[0], qmax));
   const float s = bf2f(sb);
   if (threadIdx.x == 0) scales[pr] = sb;
-  int8_t* out = static_cast<int8_t*>(dst) + (size_t)pr * cols;
-  for (int k = threadIdx.x; k < cols; k += blockDim.x) {
+  auto quant = [&](int k) -> int {
     float q = 0.f;
-    if (s > 0.f) q = fminf(127.f, fmaxf(-127.f, rintf(__fdiv_rn(load(k), s))));
-    out[k] = (int8_t)q;
+    if (s > 0.f) q = fminf(qmax, fmaxf(-qmax, rintf(__fdiv_rn(load(k), s))));
+    return (int)q;
+  };
+  if (dst_dtype == AMK_W_INT4) {   // byte j: element 2j in the low nibble, 2j + 1 in the high, each + 8
+    uint8_t* out = static_cast<uint8_t*>(dst) + (size_t)pr * (cols / 2);
+    for (int j = threadIdx.x; j < cols / 2; j += blockDim.x)
+      out[j] = (uint8_t)((quant(2 * j) + 8) | ((quant(2 * j + 1) + 8) << 4));
+    return;
   }
+  int8_t* out = static_cast<int8_t*>(dst) + (size_t)pr * cols;
+  for (int k = threadIdx.x; k < cols; k += blockDim.x) out[k] = (int8_t)quant(k);
 }
 
 }  // namespace dev

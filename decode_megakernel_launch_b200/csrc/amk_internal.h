@@ -157,7 +157,7 @@ struct Params {
   // model
   int L, d, Hq, Hkv, hd, ffn, V, max_seq;
   float eps;
-  int wdtype;          // AMK_W_INT8 / AMK_W_BF16
+  int wdtype;          // AMK_W_INT8 / AMK_W_BF16 / AMK_W_INT4
   int tied;
   int grid;
   const LayerPtrs* layers;     // device [L]

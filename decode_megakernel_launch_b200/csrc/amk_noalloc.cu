@@ -65,7 +65,7 @@ bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 
 std::vector<const void*> pointer_list(const amk_dims& d, const amk_weights& w) {
   std::vector<const void*> v = {w.embed, w.final_norm, w.lm_head, w.slm, w.k_cache, w.v_cache};
-  const bool i8 = d.weight_dtype == AMK_W_INT8;
+  const bool i8 = d.weight_dtype != AMK_W_BF16;   // quantised weights carry row scales
   for (int l = 0; l < d.n_layers; ++l) {
     v.insert(v.end(), {w.attn_norm[l], w.ffn_norm[l], w.wqkv[l], w.wo[l], w.wgu[l], w.wdown[l]});
     if (i8) v.insert(v.end(), {w.sqkv[l], w.so[l], w.sgu[l], w.sdown[l]});
@@ -86,7 +86,7 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
   if (rc) return rc;
   if (pos < 0 || pos >= d.max_seq || token_id < -1 || token_id >= d.vocab) return AMK_ERR_INVALID_ARG;
   const int L = d.n_layers;
-  const bool i8 = d.weight_dtype == AMK_W_INT8;
+  const bool i8 = d.weight_dtype != AMK_W_BF16;   // quantised weights carry row scales
   if (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->k_cache) || !aligned16(w->v_cache) ||
       !w->attn_norm || !w->ffn_norm || !w->wqkv || !w->wo || !w->wgu || !w->wdown)
     return AMK_ERR_INVALID_ARG;

@@ -57,24 +57,26 @@ std::string fmt(const char* f, long a = 0, long b = 0, long c = 0) {
 
 }  // namespace
 
-bool make_geom(int K, int esize, GemvGeom* g) {
+bool make_geom(int K, int wk, GemvGeom* g) {
   // Bytes per thread per row: larger groups amortise the per-slot reduction and bookkeeping over
   // more weight bytes (weight 1.0 for 32 B), smaller ones fit rows that larger ones do not divide.
   // Each candidate is scored by that efficiency times the fraction of compute warps it keeps busy.
-  int rb = K * esize;
-  if (K <= 0 || rb > kSlotBytes) return false;
+  // A thread holds at most 32 activations: 32 B of int8, 16 B of int4 or 64 B of bf16 per row.
+  const int rb = wk == AMK_W_INT4 ? K / 2 : wk == AMK_W_BF16 ? K * 2 : K;
+  const int max_bytes = wk == AMK_W_INT4 ? 16 : wk == AMK_W_BF16 ? 64 : 32;
+  const int min_bytes = wk == AMK_W_INT8 ? 2 : 4;      // bf16 and int4: at least one word per group
+  if (K <= 0 || (wk == AMK_W_INT4 && (K & 1)) || rb > kSlotBytes) return false;
   bool found = false;
   double best = -1.0;
   const int gbs[] = {64, 32, 16, 8, 4, 2};
   const double eff[] = {1.0, 1.0, 0.8, 0.65, 0.5, 0.4};
   for (int i = 0; i < 6; ++i) {
     const int gb = gbs[i];
-    if (esize == 2 && gb < 4) continue;                   // bf16: at least 2 elements per group
-    if (esize == 1 && gb > 32) continue;                  // int8: at most 32 bytes per thread per row
+    if (gb > max_bytes || gb < min_bytes) continue;
     if (rb % (gb * 32) != 0) continue;
     int W = rb / gb / 32;
     int nr = (W + kConsumerWarps - 1) / kConsumerWarps;
-    if (nr > (esize == 1 ? 32 : 64) / gb) continue;       // <= 32 activations per thread
+    if (nr > max_bytes / gb) continue;
     int wpg = W < kConsumerWarps ? W : kConsumerWarps;
     int rp = nr == 1 ? kConsumerWarps / wpg : 1;
     double bal = nr == 1 ? double(rp * wpg) / kConsumerWarps : double(W) / (nr * kConsumerWarps);
@@ -99,17 +101,20 @@ int check_dims(const amk_dims& d, std::string* msg) {
     return AMK_ERR_INVALID_ARG;
   }
   if (!(d.rms_eps >= 0.0f) || !(d.rope_theta > 0.0f)) { *msg = "rope_theta must be > 0 and rms_eps >= 0"; return AMK_ERR_INVALID_ARG; }
-  if (d.weight_dtype != AMK_W_INT8 && d.weight_dtype != AMK_W_BF16) { *msg = "weight_dtype"; return AMK_ERR_INVALID_ARG; }
+  if (d.weight_dtype != AMK_W_INT8 && d.weight_dtype != AMK_W_BF16 && d.weight_dtype != AMK_W_INT4) {
+    *msg = "weight_dtype";
+    return AMK_ERR_INVALID_ARG;
+  }
   if (d.head_dim != 64 && d.head_dim != 128) return bad("head_dim must be 64 or 128");
   if (d.n_q_heads % d.n_kv_heads) return bad("n_q_heads must be a multiple of n_kv_heads");
   if (d.n_q_heads / d.n_kv_heads > kMaxGroup) return bad("n_q_heads / n_kv_heads must be <= 4");
   int qd = d.n_q_heads * d.head_dim;
   for (int k : {d.d_model, d.ffn, qd})
     if (k % 64 || k > 16384) return bad("d_model, ffn and n_q_heads*head_dim must be multiples of 64, <= 16384");
-  int es = d.weight_dtype == AMK_W_INT8 ? 1 : 2;
+  const int wk = d.weight_dtype;
   GemvGeom g;
-  if (!make_geom(d.d_model, es, &g) || !make_geom(qd, es, &g) || !make_geom(d.ffn, es, &g) ||
-      !make_geom(d.d_model, 2, &g))
+  if (!make_geom(d.d_model, wk, &g) || !make_geom(qd, wk, &g) || !make_geom(d.ffn, wk, &g) ||
+      !make_geom(d.d_model, AMK_W_BF16, &g))
     return bad("a weight row does not fit a ring slot");
   return AMK_OK;
 }
@@ -128,12 +133,12 @@ int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::s
   if (cmax < 1) cmax = 1;
   p.kv_chunks_max = cmax;
   p.n_counters = L * CTR_PER_LAYER;
-  int es = d.weight_dtype == AMK_W_INT8 ? 1 : 2;
-  make_geom(d.d_model, es, &p.geom[0]);                           // QKV: K = d
-  make_geom(d.n_q_heads * hd, es, &p.geom[1]);                    // O:   K = Hq*hd
-  make_geom(d.d_model, es, &p.geom[2]);                           // GU:  K = d
-  make_geom(d.ffn, es, &p.geom[3]);                               // DOWN:K = ffn
-  make_geom(d.d_model, (d.tied_head || es == 2) ? 2 : 1, &p.geom[4]);  // LM: int8, or bf16 table
+  const int wk = d.weight_dtype;
+  make_geom(d.d_model, wk, &p.geom[0]);                           // QKV: K = d
+  make_geom(d.n_q_heads * hd, wk, &p.geom[1]);                    // O:   K = Hq*hd
+  make_geom(d.d_model, wk, &p.geom[2]);                           // GU:  K = d
+  make_geom(d.ffn, wk, &p.geom[3]);                               // DOWN:K = ffn
+  make_geom(d.d_model, d.tied_head ? AMK_W_BF16 : wk, &p.geom[4]);  // LM: its own dtype, or the bf16 table
 
   int qkv_rows = (d.n_q_heads + 2 * Hkv) * hd;
   auto s_qkv = split_rows(qkv_rows, 2, grid);

@@ -24,8 +24,8 @@ struct Plan {
   std::vector<int> o_rows;        // [grid * 2]: (row0, nrows) of each CTA's O rows
 };
 
-// Geometry of one GEMV with rows of K elements of `esize` bytes; returns false if unsupported.
-bool make_geom(int K, int esize, GemvGeom* g);
+// Geometry of one GEMV with rows of K elements of weight dtype `wk` (AMK_W_*); false if unsupported.
+bool make_geom(int K, int wk, GemvGeom* g);
 
 // Builds the plan. Returns AMK_OK, AMK_ERR_UNSUPPORTED or AMK_ERR_INVALID_ARG (msg says why).
 int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::string* msg);

@@ -15,10 +15,15 @@ from . import amk
 from . import synth
 
 
+def weight_kind(name: str) -> int:
+    """AMK_W_* code of a weight dtype name ("int8", "int4" or "bf16")."""
+    return {"int8": amk.AMK_W_INT8, "int4": amk.AMK_W_INT4, "bf16": amk.AMK_W_BF16}[name]
+
+
 def dims_of(cfg: synth.ModelConfig, max_seq: Optional[int] = None) -> amk.amk_dims:
     return amk.amk_dims(cfg.n_layers, cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn, cfg.vocab,
-                        max_seq or cfg.max_seq, cfg.rope_theta, cfg.rms_eps,
-                        amk.AMK_W_INT8 if cfg.weight_dtype == "int8" else amk.AMK_W_BF16, int(cfg.tied))
+                        max_seq or cfg.max_seq, cfg.rope_theta, cfg.rms_eps, weight_kind(cfg.weight_dtype),
+                        int(cfg.tied))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -35,8 +40,12 @@ def pack(role: int, dims: amk.amk_dims, src: torch.Tensor, dst_dtype: int, strea
     assert src.is_cuda and src.is_contiguous() and src.dim() == 2
     rows, cols = src.shape
     src_dt = amk.AMK_SRC_F32 if src.dtype == torch.float32 else amk.AMK_SRC_BF16
-    packed = torch.empty(rows * cols * (1 if dst_dtype == amk.AMK_W_INT8 else 2), dtype=torch.uint8, device=src.device)
-    scales = torch.empty(rows, dtype=torch.bfloat16, device=src.device) if dst_dtype == amk.AMK_W_INT8 else None
+    nbytes = amk.amk_packed_bytes(rows, cols, dst_dtype)
+    if nbytes == 0:
+        raise ValueError(f"cannot pack a [{rows}, {cols}] matrix as weight dtype {dst_dtype}")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=src.device)
+    quantised = dst_dtype != amk.AMK_W_BF16
+    scales = torch.empty(rows, dtype=torch.bfloat16, device=src.device) if quantised else None
     amk.check(amk.amk_pack_weight(role, C.byref(dims) if dims is not None else None, src.data_ptr(), src_dt, rows, cols,
                                   dst_dtype, packed.data_ptr(), _ptr(scales), stream), "amk_pack_weight")
     return packed, scales
@@ -101,7 +110,7 @@ class DeviceModel:
             keep.append(a)
             return p
 
-        i8 = self.dims.weight_dtype == amk.AMK_W_INT8
+        i8 = self.dims.weight_dtype != amk.AMK_W_BF16   # quantised: per-row scales
         wts = amk.amk_weights(
             _ptr(self.embed), arr(self.attn_norm), arr(self.ffn_norm), _ptr(self.final_norm),
             arr(self.w["qkv"]), arr(self.w["o"]), arr(self.w["gu"]), arr(self.w["down"]), _ptr(self.lm_w),

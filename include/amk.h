@@ -44,6 +44,7 @@ extern "C" {
 /* ---- enums ----------------------------------------------------------------------------------- */
 #define AMK_W_INT8   0   /* int8 weights, one bf16 scale per output row (W8A16) */
 #define AMK_W_BF16   1   /* bf16 weights, no scales */
+#define AMK_W_INT4   2   /* int4 weights, two per byte, one bf16 scale per output row (W4A16) */
 
 #define AMK_SRC_F32  0   /* packer source element type: fp32 */
 #define AMK_SRC_BF16 1   /* packer source element type: bf16 */
@@ -68,7 +69,7 @@ typedef struct amk_dims {
   int   max_seq;       /* KV cache capacity in positions (>= 1)                               */
   float rope_theta;    /* RoPE base (rotate-half form, no scaling)                            */
   float rms_eps;       /* RMSNorm epsilon                                                     */
-  int   weight_dtype;  /* AMK_W_INT8 or AMK_W_BF16 for every linear weight                   */
+  int   weight_dtype;  /* AMK_W_INT8, AMK_W_INT4 or AMK_W_BF16 for every linear weight      */
   int   tied_head;     /* 1: the LM head is the bf16 embedding table; 0: lm_head is given     */
 } amk_dims;
 
@@ -110,7 +111,8 @@ typedef struct amk_handle amk_handle;
 
 /* ---- packing --------------------------------------------------------------------------------- */
 
-/* Bytes of the packed weight buffer for `rows` x `cols` in `dst_dtype` (rows * cols * 1 or 2). */
+/* Bytes of the packed weight buffer for `rows` x `cols` in `dst_dtype` (rows * cols * 1 for int8,
+ * * 2 for bf16, / 2 for int4; int4 needs an even `cols`, else 0). */
 size_t amk_packed_bytes(int rows, int cols, int dst_dtype);
 
 /* Source row that lands in packed row `packed_row` for `role` (host-only helper, no GPU).
@@ -119,13 +121,16 @@ size_t amk_packed_bytes(int rows, int cols, int dst_dtype);
  * hold gate row i (source row i) and up row i (source row ffn + i). */
 int amk_packed_row_source(int role, const amk_dims* dims, int rows, int packed_row);
 
-/* Device-side weight packer (W8A16 quantiser / bf16 copier).
+/* Device-side weight packer (W8A16 / W4A16 quantiser, bf16 copier).
  *   src:        device, [rows, cols] row-major in `src_dtype`; for QKV the rows of Wq, Wk, Wv
  *               stacked, for GATE_UP the rows of Wgate then Wup.
  *   packed_out: device, amk_packed_bytes(rows, cols, dst_dtype) bytes, rows in the role's order.
- *   scales_out: device bf16 [rows] (packed order) for AMK_W_INT8; ignored (may be NULL) for bf16.
+ *   scales_out: device bf16 [rows] (packed order) for AMK_W_INT8 / AMK_W_INT4; ignored (may be NULL)
+ *               for bf16.
  * int8: s = bf16_rne(max|w_row| / 127), q = clamp(rint(w / s), -127, 127); s = 0, q = 0 for a row
- * whose scale rounds to 0. bf16: round-to-nearest-even of each element.
+ * whose scale rounds to 0. int4: the same with 7 in place of 127; element 2j of a row is the low
+ * nibble of byte j and element 2j + 1 the high nibble, each stored as q + 8 (1..15; 8 for q = 0).
+ * bf16: round-to-nearest-even of each element.
  * `dims` may be NULL for AMK_ROLE_PLAIN; for other roles rows/cols must match dims.
  * Asynchronous on `stream`. */
 int amk_pack_weight(int role, const amk_dims* dims, const void* src, int src_dtype, int rows, int cols,

@@ -24,10 +24,10 @@ Readings where the pages are silent (each is also listed in the design notes):
   * W8A16 quantiser: per output row, s = bf16_rne(max|w| / 127), q = clamp(rne(w / s), -127, 127);
     the scale is rounded before q is formed, so dequantisation q * s is exact in fp32. A row of
     zeros (or a scale that rounds to 0) gets s = 0, q = 0.
-  * W4A16 ("int4 (lossy, 2.42x reduced weight traffic) weight-only", technical summary, "Key
-    Contributions"): the same per-row symmetric scheme with 7 in place of 127, q in [-7, 7]. The
-    pages give no group size; per-row scales with the tied embedding left in bf16 reproduce the
-    quoted 2.42x traffic reduction over bf16 for the 1B-shaped model.
+  * W4A16 (the technical summary, "Key Contributions", lists a lossy int4 weight-only variant with
+    2.42x less weight traffic): the same per-row symmetric scheme with 7 in place of 127, q in
+    [-7, 7]. The pages give no group size; per-row scales with the tied embedding left in bf16
+    come within 1 % of that 2.42x reduction over bf16 for the 1B-shaped model (2.44x).
   * Everything is fp32 except the tensors that are stored in bf16: embedding, gains, scales,
     bf16 weights and the KV cache.
   * Attention is causal and includes the current position; scale 1/sqrt(hd); query head i reads
@@ -57,8 +57,9 @@ def bf16_round(x: torch.Tensor) -> torch.Tensor:
 
 
 def quantize_rows(w: torch.Tensor, qmax: int = 127) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Per-output-row symmetric weight quantiser: W8A16 with qmax = 127 (abstract: "int8 (W8A16)
-    megakernel"), W4A16 with qmax = 7 (technical summary, "Key Contributions": int4 weight-only).
+    """Per-output-row symmetric weight quantiser: W8A16 with qmax = 127 (the abstract's int8
+    weight-only variant), W4A16 with qmax = 7 (the int4 weight-only variant of the technical
+    summary, "Key Contributions").
 
     Returns (q int8 [rows, cols], s fp32 [rows] holding bf16 values) with
     s = bf16_rne(max|w_row| / qmax) and q = clamp(round_half_even(w / s), -qmax, qmax).

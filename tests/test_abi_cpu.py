@@ -9,7 +9,8 @@ from decode_megakernel_launch_b200 import synth
 amk = pytest.importorskip("decode_megakernel_launch_b200.amk", reason="libamk.so not built")
 from decode_megakernel_launch_b200.runtime import dims_of  # noqa: E402
 
-CONFIGS = ["tiny", "smollm135m", "llama1b", "llama8b", "llama1b_long32k"]
+CONFIGS = ["tiny", "smollm135m", "llama1b", "llama8b", "llama1b_long32k", "tiny_int4", "llama1b_int4",
+           "llama8b_int4"]
 
 
 def test_every_declared_symbol_is_exported():
@@ -22,6 +23,8 @@ def test_every_declared_symbol_is_exported():
 def test_packed_bytes():
     assert amk.amk_packed_bytes(6144, 4096, amk.AMK_W_INT8) == 6144 * 4096
     assert amk.amk_packed_bytes(6144, 4096, amk.AMK_W_BF16) == 2 * 6144 * 4096
+    assert amk.amk_packed_bytes(6144, 4096, amk.AMK_W_INT4) == 6144 * 4096 // 2
+    assert amk.amk_packed_bytes(3, 5, amk.AMK_W_INT4) == 0          # two nibbles per byte: even rows only
     assert amk.amk_packed_bytes(-1, 4, amk.AMK_W_INT8) == 0
     assert amk.amk_packed_bytes(4, 4, 7) == 0
 
@@ -56,7 +59,22 @@ def test_step_bytes_model():
     assert 7.5e9 < b < 7.8e9
     d.weight_dtype = amk.AMK_W_BF16
     assert amk.amk_step_bytes(C.byref(d), 1023) > 1.9 * b
+    d.weight_dtype = amk.AMK_W_INT4
+    assert amk.amk_step_bytes(C.byref(d), 1023) == w // 2 + scales + dm * 2 + (2 * L + 1) * dm * 2 + kv
     assert amk.amk_step_bytes(None, 0) == 0
+
+
+def test_step_bytes_int4_tied_head_stays_bf16():
+    # 1B shape, tied head: the head reads the bf16 embedding table, the layers read nibbles
+    d = dims_of(synth.preset("llama1b_int4"))
+    L, dm, ffn, V, qkv = 16, 2048, 8192, 128256, 3072
+    w = L * ((qkv + dm) * dm + 3 * ffn * dm)
+    scales = 2 * L * (qkv + dm + 2 * ffn + dm)
+    assert amk.amk_step_bytes(C.byref(d), 0) == w // 2 + scales + V * dm * 2 + dm * 2 + (2 * L + 1) * dm * 2 \
+        + 2 * L * 8 * 64 * 2
+    d8 = dims_of(synth.preset("llama1b", weight_dtype="bf16"))
+    # weight bytes fall by about the 2.42x the int4 variant is quoted with (per-row scales: 2.44x)
+    assert 2.40 < amk.amk_step_bytes(C.byref(d8), 0) / amk.amk_step_bytes(C.byref(d), 0) < 2.46
 
 
 @pytest.mark.parametrize("name", CONFIGS)
@@ -78,6 +96,16 @@ def test_unsupported_dims_rejected():
     d = dims_of(synth.preset("tiny"))
     d.head_dim = 96
     assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
+
+
+def test_int4_rows_must_be_a_multiple_of_256():
+    # the int4 GEMV reads at least one 32-bit word of nibbles per lane: rows of 256 elements
+    d = dims_of(synth.preset("tiny_int4"))
+    assert amk.plan_check(d, 148)[0] == amk.AMK_OK
+    d.ffn = 704
+    assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
+    d.weight_dtype = amk.AMK_W_INT8
+    assert amk.plan_check(d, 148)[0] == amk.AMK_OK
     d = dims_of(synth.preset("tiny"))
     d.n_q_heads = 16          # group of 8
     assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED

@@ -46,6 +46,37 @@ def test_packer_int8_bit_exact(src_dtype, shape):
     assert torch.equal(scales.cpu().float(), s_ref)
 
 
+def _unpack_int4(packed: torch.Tensor, rows: int, cols: int) -> torch.Tensor:
+    """Byte j of a row holds element 2j in its low nibble and 2j + 1 in its high one, each + 8."""
+    b = packed.cpu().view(rows, cols // 2).to(torch.int16)
+    q = torch.empty(rows, cols, dtype=torch.int16)
+    q[:, 0::2] = (b & 15) - 8
+    q[:, 1::2] = (b >> 4) - 8
+    return q.to(torch.int8)
+
+
+@pytest.mark.parametrize("src_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(37, 64), (300, 576), (8, 14336)])
+def test_packer_int4_bit_exact(src_dtype, shape):
+    amk, rt = _amk()
+    w = _edge_rows(*shape, seed=shape[0] + 1)
+    if src_dtype == "bf16":
+        w = w.to(torch.bfloat16).float()
+    src = (w if src_dtype == "f32" else w.to(torch.bfloat16)).cuda().contiguous()
+    packed, scales = rt.pack(amk.AMK_ROLE_PLAIN, None, src, amk.AMK_W_INT4)
+    torch.cuda.synchronize()
+    assert packed.numel() == shape[0] * shape[1] // 2
+    q_ref, s_ref = O.quantize_rows(w, 7)
+    assert torch.equal(_unpack_int4(packed, *shape), q_ref)
+    assert torch.equal(scales.cpu().float(), s_ref)
+
+
+def test_packer_int4_rejects_odd_rows():
+    amk, rt = _amk()
+    with pytest.raises(ValueError):
+        rt.pack(amk.AMK_ROLE_PLAIN, None, torch.ones(4, 5, device="cuda"), amk.AMK_W_INT4)
+
+
 @pytest.mark.parametrize("role", ["qkv", "gate_up"])
 def test_packer_row_order(role):
     amk, rt = _amk()
@@ -79,6 +110,24 @@ def test_tiny_megakernel_parity():
     res = run_and_compare(synth.preset("tiny"), compare_prompt=True)
     res.assert_ok()
     assert len(res.checks) == 16 + 32
+
+
+def test_tiny_int4_megakernel_parity():
+    res = run_and_compare(synth.preset("tiny_int4"), compare_prompt=True)
+    res.assert_ok()
+    assert len(res.checks) == 16 + 32
+
+
+def test_tiny_int4_unfused_equals_megakernel_bitwise():
+    amk, rt = _amk()
+    cfg = synth.preset("tiny_int4")
+    m = rt.DeviceModel(cfg)
+    _, fed_a, kept_a, _ = run_gpu_chain(m, cfg, 16, 16)
+    m.k_cache.zero_(); m.v_cache.zero_()
+    _, fed_b, kept_b, _ = run_gpu_chain(m, cfg, 16, 16, unfused=True)
+    m.close()
+    assert fed_a == fed_b
+    assert all(torch.equal(a, b) for a, b in zip(kept_a, kept_b))
 
 
 def test_tiny_unfused_equals_megakernel_bitwise():
@@ -138,6 +187,12 @@ ODD = [
     # bf16 weights, group 1 (MHA)
     synth.ModelConfig("odd_bf16", 23, 2, 192, 3, 3, 64, 320, 515, False, 1e4, prompt_len=7, decode_steps=10,
                       compare_steps=10, weight_dtype="bf16"),
+    # int4 weights with an int4 LM head, FFN of 3 x 256, odd vocab
+    synth.ModelConfig("odd_int4", 24, 3, 512, 4, 2, 64, 768, 1001, False, 1e4, prompt_len=9, decode_steps=12,
+                      compare_steps=12, weight_dtype="int4"),
+    # int4 weights with a tied (bf16) head, head_dim 128, one KV head
+    synth.ModelConfig("odd_int4_tied", 25, 2, 256, 2, 1, 128, 1280, 515, True, 5e5, prompt_len=5,
+                      decode_steps=20, compare_steps=20, weight_dtype="int4"),
 ]
 
 
@@ -215,13 +270,13 @@ def test_smollm135m_parity_every_step():
     assert len(res.checks) == 128 + 256
 
 
-@pytest.mark.parametrize("wdt", ["int8", "bf16"])
+@pytest.mark.parametrize("wdt", ["int8", "bf16", "int4"])
 def test_llama1b_parity(wdt):
     run_and_compare(synth.preset("llama1b", weight_dtype=wdt)).assert_ok()
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("wdt", ["int8", "bf16"])
+@pytest.mark.parametrize("wdt", ["int8", "bf16", "int4"])
 def test_llama8b_parity(wdt):
     run_and_compare(synth.preset("llama8b", weight_dtype=wdt)).assert_ok()
 

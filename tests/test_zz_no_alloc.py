@@ -30,7 +30,7 @@ def _weights(model, k_cache, v_cache):
         keep.append(a)
         return C.cast(a, C.POINTER(C.c_void_p))
 
-    i8 = model.dims.weight_dtype == amk.AMK_W_INT8
+    i8 = model.dims.weight_dtype != amk.AMK_W_BF16   # quantised: per-row scales
     w = amk.amk_weights(
         model.embed.data_ptr(), arr(model.attn_norm), arr(model.ffn_norm), model.final_norm.data_ptr(),
         arr(model.w["qkv"]), arr(model.w["o"]), arr(model.w["gu"]), arr(model.w["down"]),
