@@ -525,6 +525,18 @@ __device__ __forceinline__ int dot_chunk_i8(int acc, const uint32_t* w, const ui
   return acc;
 }
 
+// dp2a of two signed 16-bit halves of a with two unsigned bytes of b (low or high byte pair).
+__device__ __forceinline__ int dp2a_lo_su(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi_su(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // Vector loads of N consecutive elements (N in {2, 4, 8, 16}) into fp32 registers.
 // Vector loads of N consecutive elements of a vector written earlier in this launch by other CTAs.
 // They may allocate in L1 (the row partitions of a CTA read the same elements, and L1 merges those
@@ -580,6 +592,9 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 // rarely stay in L1 next to 226 KB of shared memory, at every task boundary.
 #ifndef AMK_INLINE_HOT
 #define AMK_INLINE_HOT 1
+#endif
+#ifndef AMK_INLINE_HOT4
+#define AMK_INLINE_HOT4 1
 #endif
 template <int WK>
 __device__ __forceinline__ int elem_of_byte(int b) { return WK == 0 ? b / 2 : WK == 1 ? b : b * 2; }
@@ -750,6 +765,19 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
                     // nibbles stored as q + 8: dot(a, u) - 8 * sum(a) = dot(a, q), exact in int32
                     const uint32_t* a4 = &ah[(j * NP + c) * PE / 2];
                     int acc = 0;
+#if AMK_I4_NOSHIFT
+                    // high nibbles stay in place (16 u, u < 16, as unsigned bytes) in their own sum
+                    int acc16 = 0;
+#pragma unroll
+                    for (int k = 0; k < WPP; ++k) {
+                      const uint32_t lo = w[k] & 0x0f0f0f0fu, hi = w[k] & 0xf0f0f0f0u;
+                      acc = __dp2a_lo((int)a4[4 * k + 0], (int)lo, acc);
+                      acc = __dp2a_hi((int)a4[4 * k + 1], (int)lo, acc);
+                      acc16 = dp2a_lo_su(a4[4 * k + 2], hi, acc16);
+                      acc16 = dp2a_hi_su(a4[4 * k + 3], hi, acc16);
+                    }
+                    acc += acc16 >> 4;   // a multiple of 16: the shift is exact
+#else
 #pragma unroll
                     for (int k = 0; k < WPP; ++k) {
                       const uint32_t lo = w[k] & 0x0f0f0f0fu, hi = (w[k] >> 4) & 0x0f0f0f0fu;
@@ -758,6 +786,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
                       acc = __dp2a_lo((int)a4[4 * k + 2], (int)hi, acc);
                       acc = __dp2a_hi((int)a4[4 * k + 3], (int)hi, acc);
                     }
+#endif
                     acc -= 8 * sa[j * NP + c];
                     v = fmaf((float)acc, asc[j * NP + c], v);
                   } else {
@@ -891,7 +920,7 @@ __device__ __noinline__ uint32_t gemv_task(const Params& p, const Task t, uint32
 template <int WK, int GB>
 __device__ __forceinline__ uint32_t gemv_nr(const Params& p, const Task& t, uint32_t it, int token,
                                             unsigned long long* tr, int nr) {
-  constexpr int NRMAX = (WK == 0 ? 64 : WK == 1 ? 32 : 16) / GB;
+  constexpr int NRMAX = (WK == 0 ? 64 : WK == 1 ? 32 : AMK_I4_MAX_GB) / GB;
   if constexpr (NRMAX <= 1) {
     return gemv_task<WK, GB, 1>(p, t, it, token, tr);
   } else {
@@ -1257,7 +1286,14 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
         }
       } else if (wk == AMK_W_INT4) {
         switch (g.gb) {
-          case 16: it = gemv_nr<2, 16>(p, t, it, token, tr, g.nr); break;
+#if AMK_I4_MAX_GB >= 32
+          case 32: it = gemv_nr<2, 32>(p, t, it, token, tr, g.nr); break;
+#endif
+          case 16:
+#if AMK_INLINE_HOT4
+            if (g.nr <= 1) { it = gemv_body<2, 16, 1>(p, t, it, token, tr); break; }
+#endif
+            it = gemv_nr<2, 16>(p, t, it, token, tr, g.nr); break;
           case 8: it = gemv_nr<2, 8>(p, t, it, token, tr, g.nr); break;
           default: it = gemv_nr<2, 4>(p, t, it, token, tr, g.nr); break;
         }

@@ -76,6 +76,14 @@ constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV t
 #ifndef AMK_NB32
 #define AMK_NB32 4
 #endif
+// Largest int4 group (bytes of nibbles per thread per row): 16 B = 32 elements, 32 B = 64.
+#ifndef AMK_I4_MAX_GB
+#define AMK_I4_MAX_GB 16
+#endif
+// int4 high nibbles: masked in place and met with an unsigned-byte dp2a (1) or shifted down (0).
+#ifndef AMK_I4_NOSHIFT
+#define AMK_I4_NOSHIFT 1
+#endif
 constexpr int kMaxGroup        = 4;                        // Hq / Hkv supported
 constexpr int kAuxBytes        = 8 * kMaxGroup * (128 + 2) * 4;   // attention cross-warp tree
 constexpr int kRingBytes       = kSlots * kSlotBytes;

@@ -63,7 +63,7 @@ bool make_geom(int K, int wk, GemvGeom* g) {
   // Each candidate is scored by that efficiency times the fraction of compute warps it keeps busy.
   // A thread holds at most 32 activations: 32 B of int8, 16 B of int4 or 64 B of bf16 per row.
   const int rb = wk == AMK_W_INT4 ? K / 2 : wk == AMK_W_BF16 ? K * 2 : K;
-  const int max_bytes = wk == AMK_W_INT4 ? 16 : wk == AMK_W_BF16 ? 64 : 32;
+  const int max_bytes = wk == AMK_W_INT4 ? AMK_I4_MAX_GB : wk == AMK_W_BF16 ? 64 : 32;
   const int min_bytes = wk == AMK_W_INT8 ? 2 : 4;      // bf16 and int4: at least one word per group
   if (K <= 0 || (wk == AMK_W_INT4 && (K & 1)) || rb > kSlotBytes) return false;
   bool found = false;
