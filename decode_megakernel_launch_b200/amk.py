@@ -11,7 +11,9 @@ import os
 import re
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libamk.so")
+# AMK_LIB may name a variant build of the same library (build.build_variant: other compile-time
+# knobs, same ABI); the default is the in-tree libamk.so.
+LIB_PATH = os.environ.get("AMK_LIB") or os.path.join(_PKG, "libamk.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "amk.h")
 
 if not os.path.exists(LIB_PATH):
