@@ -83,12 +83,6 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.volatile.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -179,47 +173,19 @@ __device__ bool spin_counter(const Params& p, int ctr, uint32_t target) {
   if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
   if (ld_volatile(p.abort_flag)) return false;
   const uint64_t t0 = globaltimer();
-  if constexpr (kPollWindow > 1) {
-    // kPollWindow relaxed loads in flight, staggered by kPollGapNs: a count that lands is seen about
-    // one L2 round trip later instead of up to two; the acquire fence orders what follows after it
-    uint32_t v[kPollWindow];
-#pragma unroll
-    for (int k = 0; k < kPollWindow; ++k) {
-      v[k] = ld_relaxed(c);
-      __nanosleep(kPollGapNs);
-    }
-    for (;;) {
-#pragma unroll
-      for (int k = 0; k < kPollWindow; ++k) {
-        if ((int32_t)(v[k] - target) >= 0) {
-          fence_acq_rel_gpu();
-          return true;
-        }
-        v[k] = ld_relaxed(c);
-        __nanosleep(kPollGapNs);
-      }
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(20);
+    if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
+    if ((it & 15) == 0) {
       if (ld_volatile(p.abort_flag)) return false;
       if (globaltimer() - t0 > p.timeout_ns) {
         raise_abort(p, (1u << 16) | (uint32_t)ctr);
         return false;
       }
     }
-  } else {
-    for (uint32_t it = 1;; ++it) {
-      __nanosleep(20);
-      if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
-      if ((it & 15) == 0) {
-        if (ld_volatile(p.abort_flag)) return false;
-        if (globaltimer() - t0 > p.timeout_ns) {
-          raise_abort(p, (1u << 16) | (uint32_t)ctr);
-          return false;
-        }
-      }
-    }
   }
 }
 
-// All compute threads call this; thread 0 waits, then the compute barrier publishes it.
 // All compute threads call this; thread 0 waits, then the compute barrier publishes it.
 __device__ __forceinline__ void wait_counter(const Params& p, int ctr, uint32_t mult) {
   if (threadIdx.x == 0) spin_counter(p, ctr, p.epoch * mult);

@@ -52,18 +52,9 @@ constexpr int kInflight        = AMK_INFLIGHT;             // outstanding copies
 #ifndef AMK_PF_STALL_NS
 #define AMK_PF_STALL_NS 200
 #endif
-// Counter waits keep this many polling loads in flight, one issued every kPollGapNs.
-#ifndef AMK_POLL_WINDOW
-#define AMK_POLL_WINDOW 1
-#endif
-#ifndef AMK_POLL_GAP_NS
-#define AMK_POLL_GAP_NS 200
-#endif
 constexpr int kPfItems = AMK_PF_ITEMS;
 constexpr unsigned kPfGapNs = AMK_PF_GAP_NS;
 constexpr unsigned kStallNs = AMK_PF_STALL_NS;
-constexpr int kPollWindow = AMK_POLL_WINDOW;
-constexpr unsigned kPollGapNs = AMK_POLL_GAP_NS;
 static_assert(kInflight >= 1 && kInflight <= kSlots, "ring in-flight bound");
 static_assert(kSlotBytes % 256 == 0 && kSlotBytes >= 32768, "ring slot holds a 32 KB weight row");
 constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block

@@ -41,7 +41,7 @@ def _weights(model, k_cache, v_cache):
     return w, keep
 
 
-@pytest.mark.parametrize("name", ["tiny", "smollm135m"])
+@pytest.mark.parametrize("name", ["tiny", "smollm135m", "tiny_int4"])
 def test_noalloc_matches_decode_step_on_two_calls(name):
     from decode_megakernel_launch_b200 import amk
     from decode_megakernel_launch_b200.runtime import DeviceModel
