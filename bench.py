@@ -179,6 +179,23 @@ def run_reference(args, cfg, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's value: a replica job ends with its slowest rank, so device-timed
+    regions are reduced with MAX (identity without an initialised process group of > 1 rank)."""
+    import torch
+    import torch.distributed as td
+    if not (td.is_available() and td.is_initialized()) or td.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps_per_rank: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * steps_per_rank / (max_ms / 1000.0)
+
+
 def run_gpu(args, cfg, rank, world, local_rank):
     import ctypes as C
     import torch
@@ -231,11 +248,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
     rc, detail = model.status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} detail {detail:#x}")
-    if dist:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-    value = world * args.steps / (elapsed_ms / 1000.0)
+    elapsed_ms = max_over_ranks(elapsed_ms, "cuda")
+    value = job_throughput(world, args.steps, elapsed_ms)
 
     bytes_steps = [model.step_bytes(pos_of(args.warmup + k)) for k in range(args.steps)]
     avg_bytes = sum(bytes_steps) / len(bytes_steps)
@@ -269,11 +283,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     wall_e2e = time.perf_counter() - w0
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * k_e2e / (e2e_ms / 1000.0)
+    e2e_ms = max_over_ranks(e2e_ms, "cuda")
+    e2e_value = job_throughput(world, k_e2e, e2e_ms)
 
     # ---- op-per-kernel ablation (same routines, one kernel per op), eager and CUDA-graph replay ----
     k_abl = min(args.steps, 32)
