@@ -322,6 +322,21 @@ def run_gpu(args, cfg, rank, world, local_rank):
         graph_ms = f"unavailable: {type(e).__name__}"
     info = model.plan_info()
 
+    # ---- one traced step, outside every timed region: what each op adds to the critical path ----
+    try:
+        from decode_megakernel_launch_b200.runtime import stage_breakdown
+        model.close()
+        model._create(dict(trace=1, **(dict(kv_block=args.kv_block) if args.kv_block else {})))
+        model.next_token.fill_(first_tok)
+        for k in range(3):
+            model.step(-1 if k else first_tok, pos_of(k))
+        bd = stage_breakdown(model.trace())
+        stages = {"us": {k: round(v, 2) for k, v in bd["us"].items()}, "span_us": round(bd["span_us"], 2),
+                  "position": pos_of(2), "what": "critical-path microseconds per op of one traced step "
+                  "(%globaltimer: a stage adds the time from the previous stage's last CTA to its own)"}
+    except Exception as e:  # diagnostics only
+        stages = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, secs, sample, cores = oracle_tokens_per_s(cfg)
@@ -347,7 +362,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
                        "smem_bytes": info.smem_bytes, "l2": "weights+KV per step far exceed the 126 MB L2; no flush",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "p50_ms": srt[len(srt) // 2], "p99_ms": srt[min(len(srt) - 1, int(0.99 * len(srt)))],
-            "bytes_per_step": avg_bytes, "achieved_gbs": achieved,
+            "bytes_per_step": avg_bytes, "achieved_gbs": achieved, "stage_us": stages,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "peak_source": peak_src,
                          "spec_frac": achieved / 8000.0},

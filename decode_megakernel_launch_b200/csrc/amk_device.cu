@@ -105,6 +105,17 @@ __device__ __forceinline__ void ffma2(unsigned long long& acc, float lo, float h
       : "+l"(acc)
       : "f"(lo), "f"(hi), "f"(a0), "f"(a1));
 }
+// (o0, o1) += p * (v0, v1) as one packed fp32 FMA.
+__device__ __forceinline__ void ffma2_pair(float& o0, float& o1, float p, float v0, float v1) {
+  asm("{\n\t.reg .b64 ov, pv, vv;\n\t"
+      "mov.b64 ov, {%0, %1};\n\t"
+      "mov.b64 pv, {%2, %2};\n\t"
+      "mov.b64 vv, {%3, %4};\n\t"
+      "fma.rn.f32x2 ov, pv, vv, ov;\n\t"
+      "mov.b64 {%0, %1}, ov;\n\t}"
+      : "+f"(o0), "+f"(o1)
+      : "f"(p), "f"(v0), "f"(v1));
+}
 __device__ __forceinline__ float f2sum(unsigned long long v) {
   float lo, hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
@@ -997,14 +1008,24 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
   bar_compute();
 
   float m[HW], ls[HW], o[HW][8];
+  float qr[HW][8];   // this lane's 8 query elements of each of its heads, for the whole task
+  const int g0 = hg * HW;                               // first query head of this warp's group
 #pragma unroll
   for (int g = 0; g < HW; ++g) {
     m[g] = -CUDART_INF_F;
     ls[g] = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
+    if (in_group && g0 + g < G) {
+      const float4 q0 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8);
+      const float4 q1 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8 + 4);
+      qr[g][0] = q0.x; qr[g][1] = q0.y; qr[g][2] = q0.z; qr[g][3] = q0.w;
+      qr[g][4] = q1.x; qr[g][5] = q1.y; qr[g][6] = q1.z; qr[g][7] = q1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qr[g][e] = 0.f;
+    }
   }
-  const int g0 = hg * HW;                               // first query head of this warp's group
 
   const size_t head_off = ((size_t)l * p.Hkv + h) * p.max_seq;
   for (int blk = cb; blk < ce; blk += NPS, ++it) {
@@ -1029,46 +1050,61 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
       for (int base = 0; base < n; base += WPH * PPW) {
         const int j = base + wi * PPW + sw;
         const bool valid = j < n;
+        // scores of this sub-warp's position for the warp's heads: packed fp32 FMAs over the
+        // lane's 8 elements, then a sum over the LPP lanes of the position
         float sc[HW];
         {
           const uint4 kw = valid ? *reinterpret_cast<const uint4*>(kb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
           const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+          float a[HW];
 #pragma unroll
           for (int g = 0; g < HW; ++g) {
-            float a = 0.f;
-            if (g0 + g < G) {
-              const float4 q0 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8);
-              const float4 q1 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8 + 4);
-              a = fmaf(q0.x, bf_lo(kk[0]), a);
-              a = fmaf(q0.y, bf_hi(kk[0]), a);
-              a = fmaf(q0.z, bf_lo(kk[1]), a);
-              a = fmaf(q0.w, bf_hi(kk[1]), a);
-              a = fmaf(q1.x, bf_lo(kk[2]), a);
-              a = fmaf(q1.y, bf_hi(kk[2]), a);
-              a = fmaf(q1.z, bf_lo(kk[3]), a);
-              a = fmaf(q1.w, bf_hi(kk[3]), a);
-            }
+            unsigned long long acc2 = 0ull;
 #pragma unroll
-            for (int off = 1; off < LPP; off <<= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-            sc[g] = a;
+            for (int q = 0; q < 4; ++q) ffma2(acc2, bf_lo(kk[q]), bf_hi(kk[q]), qr[g][2 * q], qr[g][2 * q + 1]);
+            a[g] = f2sum(acc2);
+          }
+          if constexpr (HW == 2) {
+            // both heads in one butterfly: the first exchange leaves head 0's pair sums on the lanes
+            // whose LPP/2 bit is clear and head 1's on the others, the rest reduce within each half
+            const bool up = cl & (LPP / 2);
+            float k = up ? a[1] : a[0];
+            k += __shfl_xor_sync(0xffffffffu, up ? a[0] : a[1], LPP / 2);
+#pragma unroll
+            for (int off = LPP / 4; off >= 1; off >>= 1) k += __shfl_xor_sync(0xffffffffu, k, off);
+            const float other = __shfl_xor_sync(0xffffffffu, k, LPP / 2);
+            sc[0] = up ? other : k;
+            sc[1] = up ? k : other;
+          } else {
+#pragma unroll
+            for (int g = 0; g < HW; ++g) {
+              float k = a[g];
+#pragma unroll
+              for (int off = 1; off < LPP; off <<= 1) k += __shfl_xor_sync(0xffffffffu, k, off);
+              sc[g] = k;
+            }
           }
         }
-        if (valid) {
-          const uint4 vw = *reinterpret_cast<const uint4*>(vb + (size_t)j * HD * 2 + cl * 16);
-          const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
+        // online softmax per sub-warp; o and l are rescaled only in steps where some lane's
+        // maximum rises (warp vote), which after the first positions is rare
+        const uint4 vw = valid ? *reinterpret_cast<const uint4*>(vb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
+        const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
 #pragma unroll
-          for (int g = 0; g < HW; ++g) {
-            if (g0 + g < G) {
-              const float mn = fmaxf(m[g], sc[g]);
-              const float cr = exp2_scale(m[g], mn), pe = fast_exp2(sc[g] - mn);
-              ls[g] = ls[g] * cr + pe;
+        for (int g = 0; g < HW; ++g) {
+          if (g0 + g < G) {
+            const bool rise = valid && sc[g] > m[g];
+            if (__any_sync(0xffffffffu, rise)) {
+              const float mn = rise ? sc[g] : m[g];
+              const float cr = exp2_scale(m[g], mn);
+              ls[g] *= cr;
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                o[g][2 * q] = fmaf(o[g][2 * q], cr, pe * bf_lo(vv[q]));
-                o[g][2 * q + 1] = fmaf(o[g][2 * q + 1], cr, pe * bf_hi(vv[q]));
-              }
+              for (int e = 0; e < 8; ++e) o[g][e] *= cr;
               m[g] = mn;
             }
+            const float pe = valid ? fast_exp2(sc[g] - m[g]) : 0.f;
+            ls[g] += pe;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ffma2_pair(o[g][2 * q], o[g][2 * q + 1], pe, bf_lo(vv[q]), bf_hi(vv[q]));
           }
         }
       }

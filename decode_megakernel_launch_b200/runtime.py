@@ -164,3 +164,36 @@ class DeviceModel:
             self.close()
         except Exception:
             pass
+
+
+OP_NAMES = {amk.AMK_OP_QKV: "qkv", amk.AMK_OP_ATTN: "attn", amk.AMK_OP_O: "o", amk.AMK_OP_GU: "gu",
+            amk.AMK_OP_DOWN: "down", amk.AMK_OP_LM: "lm"}
+
+
+def stage_breakdown(trace) -> dict:
+    """Critical-path time of each op over one traced step, from `DeviceModel.trace()` records.
+
+    A stage (op, layer) ends when its last CTA is done; stages end in dependency order, so the time
+    from one stage's end to the next stage's end is what that stage adds to the step. Returns
+    {"us": {op name: summed microseconds}, "span_us": first wait-start to the last stage end,
+    "stages": number of stages}.
+    """
+    import numpy as np
+    tr = np.asarray(trace, dtype=np.uint64)
+    tr = tr[tr[:, 3] > 0]
+    if len(tr) == 0:
+        return {"us": {}, "span_us": 0.0, "stages": 0}
+    op = (tr[:, 0] >> np.uint64(32)).astype(np.int64)
+    layer = ((tr[:, 0] >> np.uint64(16)) & np.uint64(0xFFFF)).astype(np.int64)
+    start = int(tr[:, 1].min())
+    ends = {}
+    for o, l, t in zip(op, layer, tr[:, 3].astype(np.int64)):
+        key = (int(o), int(l))
+        ends[key] = max(ends.get(key, 0), int(t))
+    out = {name: 0.0 for name in OP_NAMES.values()}
+    prev = start
+    for key, t in sorted(ends.items(), key=lambda kv: kv[1]):
+        out[OP_NAMES.get(key[0], str(key[0]))] = out.get(OP_NAMES.get(key[0], str(key[0])), 0.0) + (t - prev) / 1e3
+        prev = max(prev, t)
+    return {"us": out, "span_us": (prev - start) / 1e3, "stages": len(ends)}
+

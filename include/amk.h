@@ -231,8 +231,16 @@ int amk_plan_check(const amk_dims* dims, int grid, int mutation, char* msg, int 
 /* ---- tracing --------------------------------------------------------------------------------- */
 
 /* With options.trace = 1, every CTA records (task, wait-start, wait-end, done) %globaltimer
- * stamps of the last step. Copies up to `max_records` records of 4 uint64 each into the host
- * buffer `out` (synchronizes the device) and returns how many were written, or a negative code. */
+ * stamps (ns) of the last step. Copies up to `max_records` records of 4 uint64 each into the host
+ * buffer `out` (synchronizes the device) and returns how many were written, or a negative code.
+ * Record r of CTA b is at index b * (max tasks per CTA) + r; unused records are zero. The task word
+ * holds (op << 32) | (layer << 16) | (index of the task in its CTA's list), op one of: */
+#define AMK_OP_QKV  1   /* RMSNorm -> QKV GEMV -> RoPE -> K/V append                         */
+#define AMK_OP_ATTN 2   /* attention of one KV head over one KV chunk (+ the head's merge)    */
+#define AMK_OP_O    3   /* O GEMV + residual                                                  */
+#define AMK_OP_GU   4   /* RMSNorm -> gate/up GEMV -> SwiGLU                                  */
+#define AMK_OP_DOWN 5   /* down GEMV + residual                                               */
+#define AMK_OP_LM   6   /* final RMSNorm -> LM head -> logits + argmax                        */
 int amk_trace_read(amk_handle* h, uint64_t* out, int max_records);
 
 #ifdef __cplusplus

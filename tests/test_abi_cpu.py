@@ -130,3 +130,33 @@ def test_argument_errors_before_any_launch():
     assert amk.amk_pack_weight(amk.AMK_ROLE_QKV, C.byref(d), 16, 0, 100, 256, 0, 16, 16, None) == amk.AMK_ERR_INVALID_ARG
     assert amk.amk_pack_weight(amk.AMK_ROLE_PLAIN, None, 16, 0, 4, 4, 0, 16, None, None) == amk.AMK_ERR_INVALID_ARG
     assert amk.amk_trace_read(None, None, 0) == amk.AMK_ERR_INVALID_ARG
+
+
+def test_trace_op_codes_match_the_kernel():
+    import os
+    import re
+    text = open(os.path.join(os.path.dirname(amk.HEADER), "..", "decode_megakernel_launch_b200", "csrc",
+                             "amk_internal.h")).read()
+    enum = {m.group(1): int(m.group(2)) for m in re.finditer(r"\bOP_(\w+)\s*=\s*(\d+)", text)}
+    for name in ("QKV", "ATTN", "O", "GU", "DOWN", "LM"):
+        assert getattr(amk, "AMK_OP_" + name) == enum[name], name
+
+
+def test_stage_breakdown_of_a_synthetic_trace():
+    import numpy as np
+    from decode_megakernel_launch_b200.runtime import stage_breakdown
+
+    def rec(op, layer, ti, t0, t1, t2):
+        return [(op << 32) | (layer << 16) | ti, t0, t1, t2]
+    # two CTAs, one layer: QKV ends at 3000 ns (slowest CTA), ATTN at 7000, O 9000, GU 15000, DOWN
+    # 18000, LM 21000; the step starts at 1000 (first wait-start); one unused (zero) record
+    tr = np.array([rec(1, 0, 0, 1000, 1500, 2500), rec(1, 0, 0, 1200, 1600, 3000),
+                   rec(2, 0, 1, 3100, 3200, 7000), rec(2, 0, 1, 3000, 3300, 5000),
+                   rec(3, 0, 2, 7000, 7100, 9000), rec(4, 0, 3, 9000, 9100, 15000),
+                   rec(5, 0, 4, 15000, 15100, 18000), rec(6, 0, 5, 18000, 18100, 21000),
+                   [0, 0, 0, 0]], dtype=np.uint64)
+    bd = stage_breakdown(tr)
+    assert bd["stages"] == 6
+    assert bd["us"] == {"qkv": 2.0, "attn": 4.0, "o": 2.0, "gu": 6.0, "down": 3.0, "lm": 3.0}
+    assert bd["span_us"] == 20.0 == sum(bd["us"].values())
+    assert stage_breakdown(np.zeros((3, 4), dtype=np.uint64))["stages"] == 0

@@ -259,6 +259,9 @@ def test_trace_records_every_task():
     done = tr[tr[:, 3] > 0]
     assert len(done) == info.n_tasks
     assert (done[:, 3] >= done[:, 1]).all()
+    bd = rt.stage_breakdown(tr)
+    assert bd["stages"] == 5 * cfg.n_layers + 1
+    assert bd["span_us"] > 0 and abs(sum(bd["us"].values()) - bd["span_us"]) < 1e-6
 
 
 # ---------------------------------------------------------------------------------------------
