@@ -32,6 +32,7 @@ import argparse
 import json
 import os
 import re
+import shutil
 import subprocess
 import sys
 import tempfile
@@ -253,18 +254,20 @@ def sweep(knobs: List[Tuple[str, List[int]]], cfg_name: str, steps: int = 100, w
           check_steps: int = 8) -> dict:
     """Full search; returns the report (also what `--out` writes)."""
     tmp = tempfile.mkdtemp(prefix="amk_sweep_")
-    cands = single_candidates(knobs)
-    results, ref = evaluate(cands, cfg_name, steps, warmup, check_steps, tmp)
-    if results[0].get("ms") is None or not results[0].get("correct"):
-        raise RuntimeError(f"the default configuration failed: {results[0]}")
-    decide(results)
-    comb = combined_candidate(results)
-    if comb is not None:
-        # time the default again beside the combination, so both share one measurement window
-        again, _ = evaluate([{"runtime": {}, "compile": {}}, comb], cfg_name, steps, warmup, check_steps, tmp, ref)
-        both = [again[0], again[1]]
-        decide(both)
-        results.append(dict(both[1], combined=True, default_ms_same_run=again[0]["ms"]))
+    try:
+        cands = single_candidates(knobs)
+        results, ref = evaluate(cands, cfg_name, steps, warmup, check_steps, tmp)
+        if results[0].get("ms") is None or not results[0].get("correct"):
+            raise RuntimeError(f"the default configuration failed: {results[0]}")
+        decide(results)
+        comb = combined_candidate(results)
+        if comb is not None:
+            # time the default again beside the combination, so both share one measurement window
+            again, _ = evaluate([{"runtime": {}, "compile": {}}, comb], cfg_name, steps, warmup, check_steps, tmp, ref)
+            decide(again)
+            results.append(dict(again[1], combined=True, default_ms_same_run=again[0]["ms"]))
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
     kept = [r for r in results if r.get("keep")]
     best = min(kept, key=lambda r: r["ms"] / (r.get("default_ms_same_run") or results[0]["ms"])) if kept else None
     return {"config": cfg_name, "steps": steps, "warmup": warmup, "check_steps": check_steps,
