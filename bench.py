@@ -142,13 +142,23 @@ class OracleSample:
 
 
 def oracle_tokens_per_s(cfg, reps: int = 3):
+    """(tokens/s on all host threads, seconds spent, sample description, threads, tokens/s on one
+    thread from a single 1- and 2-layer step)."""
+    import torch
     t_all = time.time()
     smp = OracleSample(cfg)
     smp.step(1), smp.step(2)                               # warm-up
     t1 = min(smp.step(1) for _ in range(reps))
     t2 = min(smp.step(2) for _ in range(reps))
     t_token = t1 + (cfg.n_layers - 1) * max(t2 - t1, 0.0)
-    return 1.0 / t_token, time.time() - t_all, smp.describe(2 * reps), smp.threads
+    n = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        s1, s2 = smp.step(1), smp.step(2)
+    finally:
+        torch.set_num_threads(n)
+    one = 1.0 / (s1 + (cfg.n_layers - 1) * max(s2 - s1, 0.0))
+    return 1.0 / t_token, time.time() - t_all, smp.describe(2 * reps), smp.threads, one
 
 
 # ------------------------------------------------------------------------------------------------
@@ -339,9 +349,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, secs, sample, cores = oracle_tokens_per_s(cfg)
+        tps, secs, sample, cores, one = oracle_tokens_per_s(cfg)
         cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
-               "seconds": round(secs, 1)}
+               "seconds": round(secs, 1), "one_thread": {"value": one, "unit": "tokens/s", "cores": 1}}
 
     traffic = _dram_traffic(cfg.name, avg_bytes)
     comparator = None

@@ -1,0 +1,31 @@
+"""bench.py pieces that need no GPU: the CPU baseline and the reference arm's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+from decode_megakernel_launch_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_oracle_baseline_reports_all_threads_and_one():
+    tps, secs, sample, cores, one = bench.oracle_tokens_per_s(synth.preset("tiny"), reps=1)
+    assert tps > 0 and one > 0 and cores >= 1 and secs > 0
+    assert "tiny-shaped" in sample and "1 and 2 layers" in sample
+
+
+def test_reference_arm_prints_one_contract_line():
+    p = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny", "--steps", "2",
+                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["steps"] == 2 and d["warmup"] == 3 and d["higher_is_better"] is True
+    assert d["metric"] == bench.metric_for(synth.preset("tiny"))
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"]
