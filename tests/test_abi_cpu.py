@@ -160,3 +160,16 @@ def test_stage_breakdown_of_a_synthetic_trace():
     assert bd["us"] == {"qkv": 2.0, "attn": 4.0, "o": 2.0, "gu": 6.0, "down": 3.0, "lm": 3.0}
     assert bd["span_us"] == 20.0 == sum(bd["us"].values())
     assert stage_breakdown(np.zeros((3, 4), dtype=np.uint64))["stages"] == 0
+
+
+def test_step_byte_model_reproduces_the_pages_ratios():
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_ratios.json")))
+    b8 = amk.amk_step_bytes(C.byref(dims_of(synth.preset("llama1b"))), 0)
+    b16 = amk.amk_step_bytes(C.byref(dims_of(synth.preset("llama1b", weight_dtype="bf16"))), 0)
+    b4 = amk.amk_step_bytes(C.byref(dims_of(synth.preset("llama1b_int4"))), 0)
+    r = g["int8_over_bf16_step_bytes"]
+    assert abs(b8 / b16 - r["value"]) <= r["tolerance"], b8 / b16
+    r = g["bf16_over_int4_weight_bytes"]
+    assert abs(b16 / b4 - r["value"]) <= r["tolerance"], b16 / b4
