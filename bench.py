@@ -28,9 +28,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 decode tokens/s (W8A16) and achieved HBM GB/s vs B200 peak"
-DTYPE_TEXT = {"int8": "w8a16 (int8 weights, f16 activations, fp32 accumulate)",
-              "int4": "w4a16 (int4 weights, f16 activations, fp32 accumulate)",
-              "bf16": "bf16 weights, fp32 activations and accumulate"}
+DTYPE_TEXT = {"int8": "w8a16: int8 weights (bf16 row scales) x int16 activations quantised per 16 elements "
+                      "(fp32 scale), exact int32 dot per 16 elements, fp32 accumulate",
+              "int4": "w4a16: int4 weights (bf16 row scales) x int16 activations quantised per 32 elements "
+                      "(fp32 scale), exact int32 dot per 32 elements, fp32 accumulate",
+              "bf16": "bf16 weights x fp32 activations, fp32 accumulate"}
 
 
 def metric_for(cfg) -> str:
@@ -108,82 +110,79 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
-# CPU baseline: the oracle as it stands on a bounded sample of the workload
+# CPU baseline: the oracle as it stands, full-depth decode steps of the workload
 
-class OracleSample:
-    """The oracle as it stands, on a bounded sample of the workload: decode steps of models with the
-    same dims but 1 and 2 layers (same KV length). A full token costs t1 + (L - 1) * (t2 - t1)."""
+class OracleDecoder:
+    """The oracle as it stands, at full depth on the workload's own shape: an OracleModel (weights held
+    as int8 / int4 codes plus scales and dequantised per use), a KV cache filled like the GPU's
+    (the seeded prefill, or the prompt in one batched causal pass), then greedy decode steps at the
+    workload's positions, cycling through its decode span like the GPU bench."""
 
     def __init__(self, cfg):
         import torch
         from oracle import llama_decode as O
-        self.O = O
-        self.cfg = cfg
+        from decode_megakernel_launch_b200 import synth
+        t0 = time.time()
+        self.O, self.cfg = O, cfg
         self.threads = torch.get_num_threads()
-        self.models = {}
-        for nl in (1, 2):
-            c = cfg.with_(n_layers=nl)
-            om = O.OracleModel(c, keep_dequantized=False)
-            kv = O.OracleKV(c, max_seq=c.prefill_len + c.prompt_len + 2)
-            kv.prefill_synthetic()
-            self.models[nl] = (om, kv, c.prefill_len + c.prompt_len)
+        self.model = O.OracleModel(cfg, keep_dequantized=False)
+        self.kv = O.OracleKV(cfg)
+        self.start = cfg.prefill_len + cfg.prompt_len
+        if cfg.prefill_len:
+            self.kv.prefill_synthetic()
+            self.token = synth.first_decode_token(cfg)
+        else:
+            ids = synth.prompt_ids(cfg)
+            self.token = O.argmax_lowest(O.full_forward(self.model, ids, kv_out=self.kv)[-1])
+        self.k = 0
+        self.setup_s = time.time() - t0
 
-    def step(self, nl: int) -> float:
-        om, kv, pos = self.models[nl]
+    def step(self) -> float:
+        """One full decode step; returns its wall time in seconds."""
+        pos = self.start + self.k % max(1, self.cfg.decode_steps)
         t0 = time.perf_counter()
-        self.O.decode_step(om, kv, 1, pos)
-        return time.perf_counter() - t0
+        logits = self.O.decode_step(self.model, self.kv, self.token, pos)
+        dt = time.perf_counter() - t0
+        self.token = self.O.argmax_lowest(logits)
+        self.k += 1
+        return dt
 
     def describe(self, n_timed: int) -> str:
         c = self.cfg
-        return (f"oracle decode_step (torch CPU fp32, {self.threads} threads) on {c.name}-shaped models with 1 and 2 "
-                f"layers at KV length {c.prefill_len + c.prompt_len}; {n_timed} timed step(s); per-token time "
-                f"extrapolated to {c.n_layers} layers as t1 + {c.n_layers - 1}*(t2 - t1)")
+        return (f"oracle decode_step (torch CPU fp32, {self.threads} threads) on the full {c.n_layers}-layer "
+                f"{c.name}-shaped model: {n_timed} timed greedy step(s) from position {self.start} "
+                f"(model and cache set-up of {self.setup_s:.0f} s not timed)")
 
 
-def oracle_tokens_per_s(cfg, reps: int = 3):
-    """(tokens/s on all host threads, seconds spent, sample description, threads, tokens/s on one
-    thread from a single 1- and 2-layer step)."""
-    import torch
+def oracle_tokens_per_s(cfg, steps=None):
+    """(tokens/s on all host threads, seconds spent, sample description, threads): the wall time of
+    the oracle's decode steps on the steps the parity tests compare (the workload's compare_steps;
+    8B-shaped: the first 4)."""
     t_all = time.time()
-    smp = OracleSample(cfg)
-    smp.step(1), smp.step(2)                               # warm-up
-    t1 = min(smp.step(1) for _ in range(reps))
-    t2 = min(smp.step(2) for _ in range(reps))
-    t_token = t1 + (cfg.n_layers - 1) * max(t2 - t1, 0.0)
-    n = torch.get_num_threads()
-    torch.set_num_threads(1)
-    try:
-        s1, s2 = smp.step(1), smp.step(2)
-    finally:
-        torch.set_num_threads(n)
-    one = 1.0 / (s1 + (cfg.n_layers - 1) * max(s2 - s1, 0.0))
-    return 1.0 / t_token, time.time() - t_all, smp.describe(2 * reps), smp.threads, one
+    dec = OracleDecoder(cfg)
+    n = steps or max(1, cfg.compare_steps)
+    times = [dec.step() for _ in range(n)]
+    return n / sum(times), time.time() - t_all, dec.describe(n), dec.threads
 
 
 # ------------------------------------------------------------------------------------------------
 
 def run_reference(args, cfg, rank, world):
-    """The reference arm: the CPU oracle. Warm-up steps calibrate the per-layer cost (2-layer minus
-    1-layer step); each timed step is one 1-layer decode step; the reported rate is per full token."""
+    """The reference arm: the CPU oracle, W untimed and K timed full-depth decode steps of the same
+    workload on the host cores (rank 0 only)."""
     if rank != 0:
         return
-    smp = OracleSample(cfg)
-    t1s, t2s = [], []
+    dec = OracleDecoder(cfg)
     for _ in range(args.warmup):
-        t1s.append(smp.step(1))
-        t2s.append(smp.step(2))
-    t_layer = max(statistics.median(t2s) - statistics.median(t1s), 0.0)
-    timed = [smp.step(1) for _ in range(args.steps)]
-    t1 = statistics.median(timed)
-    value = 1.0 / (t1 + (cfg.n_layers - 1) * t_layer)
-    sample = smp.describe(args.steps) + "; per-layer cost calibrated over the warm-up steps"
+        dec.step()
+    timed = [dec.step() for _ in range(args.steps)]
+    value = args.steps / sum(timed)
     line = {"impl": "reference", "metric": metric_for(cfg), "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": _workload_name(cfg)},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": dec.threads, "kind": "oracle",
+                             "sample": dec.describe(args.steps)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -349,9 +348,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, secs, sample, cores, one = oracle_tokens_per_s(cfg)
+        tps, secs, sample, cores = oracle_tokens_per_s(cfg)
         cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
-               "seconds": round(secs, 1), "one_thread": {"value": one, "unit": "tokens/s", "cores": 1}}
+               "seconds": round(secs, 1)}
 
     traffic = _dram_traffic(cfg.name, avg_bytes)
     comparator = None
@@ -529,17 +528,15 @@ def run_bf16_comparator(cfg, steps, warmup):
 
 
 def _dram_traffic(workload, algorithmic_bytes):
-    """DRAM read+write bytes per launch from the committed ncu summary: its measured traffic /
-    algorithmic ratio times this launch's algorithmic bytes, or None when the summary was taken on
-    other kernel sources (or is missing)."""
-    path = os.path.join(ROOT, "profiles", "decode_kernel_dram_traffic.md")
+    """DRAM read+write bytes per launch: the measured traffic / algorithmic ratio recorded beside the
+    ncu summary (profiles/decode_kernel_dram_traffic.json) times this launch's algorithmic bytes, or
+    None when the ratio was taken on other kernel sources (or is missing)."""
     try:
-        for line in open(path):
-            if line.startswith("traffic:"):
-                kv = dict(tok.split("=", 1) for tok in line.split()[1:])
-                if kv.get("workload") == workload and kv.get("kernel") == _kernel_hash():
-                    return float(kv["ratio"]) * algorithmic_bytes
-    except (OSError, ValueError, KeyError):
+        with open(os.path.join(ROOT, "profiles", "decode_kernel_dram_traffic.json")) as f:
+            ent = json.load(f)["workloads"][workload]
+        if ent["kernel"] == _kernel_hash():
+            return float(ent["ratio"]) * algorithmic_bytes
+    except (OSError, ValueError, KeyError, TypeError):
         return None
     return None
 

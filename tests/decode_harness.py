@@ -56,9 +56,17 @@ class RunResult:
     gpu_seconds: float
     oracle_seconds: float
 
-    def assert_ok(self):
+    @property
+    def gated(self) -> int:
+        """Compared steps whose oracle top-1/top-2 margin exceeds MARGIN, i.e. whose greedy token was
+        required to match the oracle's."""
+        return sum(c.margin > MARGIN for c in self.checks)
+
+    def assert_ok(self, min_gated: int = 1):
         bad = [c for c in self.checks if not c.ok]
         assert not bad, f"{len(bad)} of {len(self.checks)} steps out of tolerance, first: {bad[0]}"
+        # a run where no step armed the token check would pass even with a broken margin or argmax
+        assert self.gated >= min_gated, f"only {self.gated} of {len(self.checks)} steps had their token checked"
 
 
 def run_gpu_chain(model, cfg: synth.ModelConfig, decode_steps: int, keep: int, unfused: bool = False,

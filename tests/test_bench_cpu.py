@@ -10,10 +10,24 @@ from decode_megakernel_launch_b200 import synth
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_oracle_baseline_reports_all_threads_and_one():
-    tps, secs, sample, cores, one = bench.oracle_tokens_per_s(synth.preset("tiny"), reps=1)
-    assert tps > 0 and one > 0 and cores >= 1 and secs > 0
-    assert "tiny-shaped" in sample and "1 and 2 layers" in sample
+def test_oracle_baseline_times_full_depth_steps():
+    tps, secs, sample, cores = bench.oracle_tokens_per_s(synth.preset("tiny"), steps=2)
+    assert tps > 0 and cores >= 1 and secs > 0
+    assert "full 2-layer tiny-shaped" in sample and "2 timed greedy step(s) from position 16" in sample
+
+
+def test_oracle_decoder_follows_the_oracle_greedy_chain():
+    # the timed steps are the oracle's own greedy chain from the prompt: same tokens as decode_step
+    from oracle import llama_decode as O
+    cfg = synth.preset("tiny")
+    dec = bench.OracleDecoder(cfg)
+    om, kv = O.OracleModel(cfg), O.OracleKV(cfg)
+    tok = O.argmax_lowest(O.full_forward(om, synth.prompt_ids(cfg), kv_out=kv)[-1])
+    assert dec.token == tok
+    for s in range(3):
+        dec.step()
+        tok = O.argmax_lowest(O.decode_step(om, kv, tok, cfg.prompt_len + s))
+        assert dec.token == tok
 
 
 def test_reference_arm_prints_one_contract_line():

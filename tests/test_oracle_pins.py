@@ -239,6 +239,50 @@ def test_argmax_lowest_on_ties():
 
 
 # ---------------------------------------------------------------------------------------------
+# The token gate. Greedy decode is exact ("Experimental Results", "Correctness & Portability" of the
+# technical summary: token-for-token agreement), and the GPU tests require the GPU's token to equal
+# the oracle's wherever the oracle's top-1 minus top-2 logit exceeds 0.1, so that margin is pinned to
+# a plain Python sort of the same float values (ties at the top give 0).
+
+def _top2_margin_py(values):
+    s = sorted((float(v) for v in values), reverse=True)
+    return s[0] - s[1]
+
+
+def _top2_cases():
+    g = torch.Generator().manual_seed(5)
+    yield torch.tensor([1.0, 3.0, 2.0, 3.0])                     # tie at the top: 0
+    yield torch.tensor([-5.0, -1.5, -9.0, -1.25])                # all negative: 0.25
+    yield torch.tensor([7.0, 7.0, 7.0])                          # all equal: 0
+    yield torch.tensor([0.0, 100.0])                             # two logits: 100
+    yield torch.tensor([2.0, 2.05, -3.0, 1.0])                   # a near tie: 0.05
+    yield torch.randn(128256, generator=g) * 3.0                # a vocabulary of the 1B / 8B shapes
+    big = torch.randn(50000, generator=g)
+    big[123], big[40000] = 9.0, 8.75                             # a clear runner-up far from the top
+    yield big
+
+
+def _top2_agrees(fn):
+    return all(math.isclose(fn(t), _top2_margin_py(t.tolist()), rel_tol=0.0, abs_tol=1e-5) for t in _top2_cases())
+
+
+def test_top2_margin_matches_a_python_sort():
+    assert _top2_agrees(O.top2_margin)
+    assert O.top2_margin(torch.tensor([1.0, 3.0, 2.0, 3.0])) == 0.0
+
+
+@pytest.mark.parametrize("fn", [
+    lambda t: float(t.max() - t.min()),                                      # top minus bottom
+    lambda t: float(torch.topk(t.abs(), 2).values[0] - torch.topk(t.abs(), 2).values[1]),   # magnitudes
+    lambda t: (lambda m: m if m > 0.1 else 0.0)(O.top2_margin(t)),           # near ties dropped
+    lambda t: (lambda u: float(u[-1] - u[-2]) if len(u) > 1 else 0.0)(torch.unique(t)),  # distinct values
+    lambda t: float(torch.sort(t).values[1] - torch.sort(t).values[0]),      # the bottom two
+], ids=["max_minus_min", "abs", "zero_near_ties", "distinct", "bottom_two"])
+def test_top2_margin_pin_catches_planted_mistakes(fn):
+    assert not _top2_agrees(fn)
+
+
+# ---------------------------------------------------------------------------------------------
 # Whole step: incremental == full causal forward; closed-form special case; HuggingFace Llama.
 
 def test_incremental_equals_full_causal_forward():
