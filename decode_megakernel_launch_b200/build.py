@@ -20,7 +20,7 @@ def _newest_source_mtime() -> float:
 # Compile-time knobs of the kernel (macros of csrc/amk_internal.h) that a variant build may set,
 # with the values the kernel's static checks and the planner accept.
 TUNABLE = {
-    "AMK_SLOT_BYTES": (32768, 49152, 65536),   # ring slot size (3 slots of 64 KB fill shared memory)
+    "AMK_SLOT_BYTES": (32768, 49152, 65536),   # ring slot size (the ring and the 64 KB input stage share 227 KB)
     "AMK_SLOTS": (2, 3, 4, 5, 6),             # ring depth (static_assert bounds the total)
     "AMK_INFLIGHT": (1, 2, 3, 4),             # outstanding bulk copies (<= slots)
     "AMK_PF_ITEMS": tuple(range(0, 17)),      # L2 warm-up items while the compute warps stall
@@ -28,6 +28,9 @@ TUNABLE = {
     "AMK_PF_STALL_NS": (100, 200, 400, 800),
     "AMK_NB32": (2, 4),                       # rows per register batch, 32-byte groups
     "AMK_I4_NOSHIFT": (0, 1),                 # int4 high nibbles in place (1) or shifted (0)
+    "AMK_CONSUMER_WARPS": (12, 15, 16),       # compute warps per CTA (16 caps registers at 96)
+    "AMK_INLINE_HOT": (0, 1),                 # the hot int8 GEMV instance inlined into the task loop
+    "AMK_INLINE_HOT4": (0, 1),                # the same for the hot int4 instance
 }
 
 

@@ -282,24 +282,23 @@ int amk_create(const amk_dims* dims, const amk_weights* w, const amk_options* op
   p.rope = rope_d;
 
   const int G = d.n_q_heads / d.n_kv_heads;
-  if ((rc = h->alloc(&p.x, d.d_model)) || (rc = h->alloc(&p.q, (size_t)d.n_q_heads * d.head_dim)) ||
-      (rc = h->alloc(&p.attn_out, (size_t)d.n_q_heads * d.head_dim)) || (rc = h->alloc(&p.act, d.ffn)) ||
+  // tagged vectors start zeroed: tag 0 never matches (epochs start at 1)
+  if ((rc = h->alloc(&p.x, d.d_model / 2)) || (rc = h->alloc(&p.xres, d.d_model)) ||
+      (rc = h->alloc(&p.qkv, (size_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim)) ||
+      (rc = h->alloc(&p.attn_out, (size_t)d.n_q_heads * d.head_dim / 2)) || (rc = h->alloc(&p.act, d.ffn / 2)) ||
       (rc = h->alloc(&p.attn_part, (size_t)d.n_kv_heads * pl.kv_chunks_max * G * (d.head_dim + 2))) ||
-      (rc = h->alloc(&p.am_val, grid)) || (rc = h->alloc(&p.am_idx, grid)) ||
+      (rc = h->alloc(&p.am, 2 * (size_t)grid)) ||
       (rc = h->alloc(&p.ctr, pl.n_counters)) || (rc = h->alloc(&p.attn_ticket, (size_t)L * d.n_kv_heads)) ||
       (rc = h->alloc(&p.am_ticket, 1)) || (rc = h->alloc(&p.abort_flag, 1)))
     return fail(rc);
   if (h->opt.trace) {
-    if ((rc = h->alloc(&p.trace, (size_t)grid * h->max_tasks_per_cta * 4))) return fail(rc);
+    if ((rc = h->alloc(&p.trace, (size_t)grid * h->max_tasks_per_cta * AMK_TRACE_WORDS))) return fail(rc);
   }
   Task* tasks_d;
   int* off_d;
-  int* orows_d;
-  if ((rc = h->upload(&tasks_d, pl.tasks)) || (rc = h->upload(&off_d, pl.off)) || (rc = h->upload(&orows_d, pl.o_rows)))
-    return fail(rc);
+  if ((rc = h->upload(&tasks_d, pl.tasks)) || (rc = h->upload(&off_d, pl.off))) return fail(rc);
   p.tasks = tasks_d;
   p.task_off = off_d;
-  p.o_rows = orows_d;
   for (const StageList& st : pl.stages) {
     DeviceStage ds{st.op, st.layer, nullptr, nullptr};
     if ((rc = h->upload(&ds.tasks, st.tasks)) || (rc = h->upload(&ds.off, st.off))) return fail(rc);
@@ -333,12 +332,12 @@ int amk_decode_step(amk_handle* h, int token_id, int pos, float* logits_out, int
   if (rc) return rc;
   Params p = h->base;
   p.epoch = ++h->epoch;
+  p.tag_epoch = p.epoch;
   p.token = token_id;
   p.pos = pos;
   p.logits = logits_out;
   p.next_token = next_token_out;
   p.sync = 1;
-  p.init_x = 1;
   cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream), true);
   return e == cudaSuccess ? AMK_OK : cuda_fail(e, "cudaLaunchCooperativeKernel");
 }
@@ -348,18 +347,17 @@ int amk_decode_step_unfused(amk_handle* h, int token_id, int pos, float* logits_
   int rc = check_step_args(h, token_id, pos, next_token_out);
   if (rc) return rc;
   Params p = h->base;
+  p.epoch = ++h->epoch;   // one tag epoch for all of this step's launches
+  p.tag_epoch = p.epoch;
   p.token = token_id;
   p.pos = pos;
   p.logits = logits_out;
   p.next_token = next_token_out;
   p.sync = 0;
   p.trace = nullptr;
-  bool first = true;
   for (const DeviceStage& st : h->stages) {
     p.tasks = st.tasks;
     p.task_off = st.off;
-    p.init_x = first ? 1 : 0;
-    first = false;
     cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream), false);
     if (e != cudaSuccess) return cuda_fail(e, "unfused launch");
   }
@@ -391,7 +389,7 @@ int amk_trace_read(amk_handle* h, uint64_t* out, int max_records) {
   int n = std::min(max_records, h->plan.grid * h->max_tasks_per_cta);
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  e = cudaMemcpy(out, h->base.trace, (size_t)n * 4 * sizeof(uint64_t), cudaMemcpyDeviceToHost);
+  e = cudaMemcpy(out, h->base.trace, (size_t)n * AMK_TRACE_WORDS * sizeof(uint64_t), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
   return n;
 }

@@ -1,6 +1,6 @@
 // Device code of libamk (sm_100a): the persistent decode kernel, its routines, and the weight packer.
 //
-// One CTA per SM, 17 warps: warp 16 is the producer, whose elected lane streams every byte this CTA
+// One CTA per SM, compute warps + 1: the last warp is the producer, whose elected lane streams every byte this CTA
 // will read (weight rows of its GEMV tasks, KV rows of its attention chunk) into a kSlots x kSlotBytes
 // shared-memory ring with cp.async.bulk, completion tracked by one mbarrier per slot; at most
 // kInflight copies are outstanding at once. The producer
@@ -10,9 +10,15 @@
 // (README summary), with dependencies carried by counters instead of grid barriers (technical
 // summary, "Methodology", Layer 0: wait -> dispatch -> signal on monotonic counters).
 //
-// Warps 0..15 compute. Every wait is bounded by a %globaltimer deadline; when one expires the CTA
-// raises a device abort flag plus a host-visible status word and every later counter wait returns
-// at once, so the launch always completes (outputs are then garbage and the handle reports it).
+// Hand-offs between CTAs carry no memory fence: every vector one CTA passes to others goes out in
+// tagged 64-bit words (see tag_of), a reader re-reads any word whose tag is not the one it expects,
+// and a stage counter, bumped with a relaxed reduction, only tells readers of a wide vector when to
+// start (a gpu-scope release fence would wait on the SM's in-flight weight copies: several
+// microseconds per stage under the full stream).
+//
+// The other warps compute. Every wait is bounded by a %globaltimer deadline; when one expires the CTA
+// raises a device abort flag plus a host-visible status word and every later wait returns at once,
+// so the launch always completes (outputs are then garbage and the handle reports it).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -77,10 +83,15 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) {
@@ -89,6 +100,51 @@ __device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) {
   return v;
 }
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void red_relaxed_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_relaxed_add(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+// Tagged pairs: {fp32 value bits (low word), tag (high word)} as one aligned 64-bit element. Loads
+// go to L2 (.cg: never a stale L1 line) on every call.
+__device__ __forceinline__ uint64_t pair_of(float v, uint32_t tag) {
+  return (uint64_t)__float_as_uint(v) | ((uint64_t)tag << 32);
+}
+__device__ __forceinline__ void st_pair(uint64_t* p, float v, uint32_t tag) {
+  asm volatile("st.global.cg.u64 [%0], %1;" ::"l"(p), "l"(pair_of(v, tag)) : "memory");
+}
+__device__ __forceinline__ void st_pair2(uint64_t* p, float a, float b, uint32_t tag) {   // 16-byte aligned
+  asm volatile("st.global.cg.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(pair_of(a, tag)), "l"(pair_of(b, tag)) : "memory");
+}
+__device__ __forceinline__ uint2 ld_pair(const uint64_t* p) {   // {value bits, tag}
+  uint64_t w;
+  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return make_uint2((uint32_t)w, (uint32_t)(w >> 32));
+}
+__device__ __forceinline__ uint4 ld_pair2(const uint64_t* p) {   // two pairs, 16-byte aligned: {v0, t0, v1, t1}
+  uint64_t a, b;
+  asm volatile("ld.global.cg.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+  return make_uint4((uint32_t)a, (uint32_t)(a >> 32), (uint32_t)b, (uint32_t)(b >> 32));
+}
+__device__ __forceinline__ bool tags_ok(uint4 v, uint32_t tag) { return v.y == tag && v.w == tag; }
+// A tagged word of two bf16 values (round to nearest even).
+__device__ __forceinline__ uint64_t bf2_word(float a, float b, uint32_t tag);
+// Two tagged words (16-byte aligned) through L1: readers use this right after an acquire poll of
+// the stage counter (which drops stale L1 lines), so the row partitions of a CTA that read the same
+// words share one L2 request.
+__device__ __forceinline__ uint4 ld_words2_ca(const uint64_t* p) {
+  uint64_t a, b;
+  asm volatile("ld.global.ca.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+  return make_uint4((uint32_t)a, (uint32_t)(a >> 32), (uint32_t)b, (uint32_t)(b >> 32));
+}
+__device__ __forceinline__ uint2 ld_word_ca(const uint64_t* p) {
+  uint64_t w;
+  asm volatile("ld.global.ca.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return make_uint2((uint32_t)w, (uint32_t)(w >> 32));
+}
 
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
 __device__ __forceinline__ uint16_t f2bf(float f) {
@@ -178,7 +234,10 @@ __device__ void raise_abort(const Params& p, uint32_t detail) {
 
 // Thread 0 of the compute warps spins until counter >= target (mod 2^32), bounded by the timeout.
 // Returns false if the wait expired or another CTA aborted (the caller then carries on: data are
-// garbage but every thread keeps the same control flow, so the launch still completes).
+// garbage but every thread keeps the same control flow, so the launch still completes). The count
+// only says when the tagged inputs are worth reading; its acquire loads (cheap: it is the writer's
+// release that waits on the SM's in-flight copies) also drop this SM's stale L1 lines, so the
+// inputs can then be read through L1.
 __device__ bool spin_counter(const Params& p, int ctr, uint32_t target) {
   const uint32_t* c = p.ctr + ctr;
   if ((int32_t)(ld_acquire(c) - target) >= 0) return true;
@@ -203,11 +262,56 @@ __device__ __forceinline__ void wait_counter(const Params& p, int ctr, uint32_t 
   bar_compute();
 }
 
-// The caller has passed a compute barrier after the task's last global store; thread 0's release
-// reduction then orders every store of the CTA before the count (release is cumulative over what
-// the barrier made visible to thread 0), pairing with the acquire load in spin_counter.
+// The caller has passed a compute barrier after the task's last tagged store. The count carries no
+// data (readers check the tags), so it needs no release: a relaxed reduction.
 __device__ __forceinline__ void signal_counter(const Params& p, int ctr) {
-  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.ctr + ctr) : "memory");
+  if (threadIdx.x == 0) red_relaxed_add(p.ctr + ctr, 1u);
+}
+
+// Re-reads, all together, the 16-byte loads (two tagged pairs each) of `v` whose bit is set in
+// `stale` until both tags of each are `tag`: the slow path of a reader that outran the writers'
+// stores (no fence orders them before the counter), one round trip per round. Bounded by the
+// timeout; after an abort it returns at once with what it read. `addr(j)` is load j's address.
+template <int N, class Addr>
+__device__ __forceinline__ void repoll2(const Params& p, uint4 (&v)[N], uint32_t stale, uint32_t tag, Addr addr) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t round = 1; stale; ++round) {
+    __nanosleep(32);
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if (stale & (1u << j)) v[j] = ld_pair2(addr(j));
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if ((stale & (1u << j)) && tags_ok(v[j], tag)) stale &= ~(1u << j);
+    if (stale && (round & 7) == 0) {
+      if (ld_volatile(p.abort_flag)) return;
+      if (globaltimer() - t0 > p.timeout_ns) {
+        raise_abort(p, 6u << 16);
+        return;
+      }
+    }
+  }
+}
+// The same for single 8-byte pairs ({value bits, tag} in x, y).
+template <int N, class Addr>
+__device__ __forceinline__ void repoll1(const Params& p, uint2 (&v)[N], uint32_t stale, uint32_t tag, Addr addr) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t round = 1; stale; ++round) {
+    __nanosleep(32);
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if (stale & (1u << j)) v[j] = ld_pair(addr(j));
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if ((stale & (1u << j)) && v[j].y == tag) stale &= ~(1u << j);
+    if (stale && (round & 7) == 0) {
+      if (ld_volatile(p.abort_flag)) return;
+      if (globaltimer() - t0 > p.timeout_ns) {
+        raise_abort(p, 6u << 16);
+        return;
+      }
+    }
+  }
 }
 
 // Bounded wait on a ring mbarrier phase. Its bound is 4x the counter bound, so a stalled counter is
@@ -361,9 +465,11 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
   int last_task = -1;
   const uint8_t *a0, *a1;
   uint32_t n0, n1;
+  bool first_item = false;
   while (next_item(p, tasks, nt, cur, a0, n0, a1, n1)) {
     if (cur.ti != last_task) {
       last_task = cur.ti;
+      first_item = true;
       prefetch_side_data(p, tasks[cur.ti], token);
     }
     const int slot = it % kSlots;
@@ -416,6 +522,10 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
       const uint32_t j = it - kInflight;
       wait_slot(p, &s.full[j % kSlots], (j / kSlots) & 1, (5u << 16) | (j % kSlots));
     }
+    if (first_item && p.trace) {   // the producer's view of the task: its first item is issued now
+      p.trace[((size_t)blockIdx.x * p.max_tasks_per_cta + cur.ti) * AMK_TRACE_WORDS + 8] = globaltimer();
+      first_item = false;
+    }
     if (n0 + n1 > 0) {
       mbar_expect_tx(&s.full[slot], n0 + n1);
       bulk_g2s(s.ring + slot * kSlotBytes, a0, n0, &s.full[slot], pol);
@@ -423,6 +533,8 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
     } else {
       mbar_arrive(&s.full[slot]);
     }
+    if (p.trace && cur.sub >= cur.end)   // the task's last item is issued
+      p.trace[((size_t)blockIdx.x * p.max_tasks_per_cta + cur.ti) * AMK_TRACE_WORDS + 9] = globaltimer();
     ++it;
   }
 }
@@ -548,6 +660,12 @@ __device__ __forceinline__ void ld_bf16_words(const uint16_t* p, uint32_t* o) { 
   }
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ uint64_t bf2_word(float a, float b, uint32_t tag) {
+  return (uint64_t)((uint32_t)f2bf(a) | ((uint32_t)f2bf(b) << 16)) | ((uint64_t)tag << 32);
+}
+__device__ __forceinline__ void st_word(uint64_t* p, uint64_t w) {
+  asm volatile("st.global.cg.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // Byte offset, inside a row, of piece c of the group that (warp column col, lane) owns. A group of
@@ -567,12 +685,6 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 // The hot GEMV instance (int8, 32-byte groups, one group per thread) is inlined into the kernel's
 // task loop: a non-inlined call saves and restores registers through local memory, whose lines
 // rarely stay in L1 next to 226 KB of shared memory, at every task boundary.
-#ifndef AMK_INLINE_HOT
-#define AMK_INLINE_HOT 1
-#endif
-#ifndef AMK_INLINE_HOT4
-#define AMK_INLINE_HOT4 1
-#endif
 template <int WK>
 __device__ __forceinline__ int elem_of_byte(int b) { return WK == 0 ? b / 2 : WK == 1 ? b : b * 2; }
 
@@ -610,58 +722,135 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
   }
   const uint16_t* gain =
       op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : op == OP_LM ? p.final_norm : nullptr;
+  float* const resid_rows = s.aux;   // residual rows (O, down) or the RoPE row (QKV)
   if (op == OP_QKV)
-    for (int i = tid; i < p.hd; i += kConsumerThreads) s.aux[i] = __ldg(p.rope + (size_t)p.pos * p.hd + i);
+    for (int i = tid; i < p.hd; i += kConsumerThreads) resid_rows[i] = __ldg(p.rope + (size_t)p.pos * p.hd + i);
 
   if (p.sync && first && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
   if (tr && tid == 0) tr[2] = globaltimer();
 
-  // ---- inputs: this thread's own elements with their RMSNorm gains and, for O / down, the
-  //      residual of the task's rows (x is final here: its last writer precedes the awaited stage),
-  //      all in one batch of loads ----
+  // ---- inputs: this thread's own elements (tagged bf16 pairs, read through L1 right after the
+  //      acquire poll; any stale word re-read) with their RMSNorm gains and, for O / down, the
+  //      residual of the task's rows (fp32 rows this CTA wrote itself), all in one batch of loads ----
   // Row partition 0 covers every input element exactly once, so its threads' squares sum to the
   // RMSNorm statistic; each warp leaves its share in misc->red and the epilogue (behind its own
   // barrier) finishes the sum, so the prologue has a single dependent L2 round trip and no barrier.
   static_assert(kMaxTaskRows <= 2 * kConsumerThreads, "two residual rows per thread");
   const bool resid = op == OP_O || op == OP_DOWN;
-  float rv0 = 0.f, rv1 = 0.f;
-  if (resid && tid < nrows) rv0 = __ldca(p.x + row0 + tid);
-  if (resid && tid + kConsumerThreads < nrows) rv1 = __ldca(p.x + row0 + tid + kConsumerThreads);
   const bool from_embed = op == OP_QKV && l == 0;
-  const float* src = op == OP_O ? p.attn_out : op == OP_DOWN ? p.act : p.x;
+  const uint32_t ep = p.tag_epoch;
+  // who wrote what: QKV(l) reads x after down(l - 1), GU(l) x after O(l), O(l) the merged attention,
+  // DOWN(l) the SwiGLU output, the LM head x after the last down
+  const uint64_t* src = op == OP_O ? p.attn_out : op == OP_DOWN ? p.act : p.x;
+  const uint32_t tag_in = op == OP_QKV ? tag_of(ep, l - 1, 1) : op == OP_LM ? tag_of(ep, p.L - 1, 1) : tag_of(ep, l, 0);
+  // the residual of O(l) is x after down(l - 1) (the embedding row for layer 0), of DOWN(l) x after O(l)
   const uint16_t* erow = p.embed + (size_t)token * p.d;
+  float rv0 = 0.f, rv1 = 0.f;
+  if (resid) {
+    const bool re = op == OP_O && l == 0;
+    if (tid < nrows) rv0 = re ? bf2f(__ldg(erow + row0 + tid)) : __ldca(p.xres + row0 + tid);
+    if (tid + kConsumerThreads < nrows)
+      rv1 = re ? bf2f(__ldg(erow + row0 + tid + kConsumerThreads)) : __ldca(p.xres + row0 + tid + kConsumerThreads);
+  }
+  // this thread's words: PE / 2 per piece (two bf16 elements each), loaded two at a time
+  constexpr int NW = NR * NP * PE / 2;          // words of the thread
+  constexpr int NL = PE >= 4 ? NW / 2 : NW;     // 16-byte loads of two words (8-byte loads of one when a piece is 2 elements)
+  uint4 wv[NL];
+  auto waddr = [&](int k) {   // address of load k: piece k / (loads per piece), its (k % ...)-th pair of words
+    constexpr int LPP = PE >= 4 ? PE / 4 : 1;
+    const int j = (k / LPP) / NP, c = (k / LPP) % NP;
+    return src + elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c)) / 2 + 2 * (k % LPP);
+  };
   float ss = 0.f;
   float xv[NR * NP * PE];
+  if (from_embed) {
 #pragma unroll
-  for (int j = 0; j < NR; ++j) {
+    for (int j = 0; j < NR; ++j) {
 #pragma unroll
-    for (int c = 0; c < NP; ++c) {
-      float* xp = &xv[(j * NP + c) * PE];
-      const int e = elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c));
-      if (ok[j]) {
-        if (from_embed) {
+      for (int c = 0; c < NP; ++c) {
+        float* xp = &xv[(j * NP + c) * PE];
+        const int e = elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c));
+        if (ok[j]) {
           uint32_t ew[PE / 2];
           ld_bf16_words<PE>(erow + e, ew);
 #pragma unroll
           for (int k = 0; k < PE / 2; ++k) { xp[2 * k] = bf_lo(ew[k]); xp[2 * k + 1] = bf_hi(ew[k]); }
         } else {
-          ld_f32_ca<PE>(src + e, xp);
-        }
-        if (norm) {
-          uint32_t gw[PE / 2];
-          ld_bf16_words<PE>(gain + e, gw);
 #pragma unroll
-          for (int k = 0; k < PE; ++k) ss = fmaf(xp[k], xp[k], ss);
-#pragma unroll
-          for (int k = 0; k < PE / 2; ++k) { xp[2 * k] *= bf_lo(gw[k]); xp[2 * k + 1] *= bf_hi(gw[k]); }
+          for (int k = 0; k < PE; ++k) xp[k] = 0.f;
         }
+      }
+    }
+  } else {
+    constexpr int LPP = PE >= 4 ? PE / 4 : 1;
+#pragma unroll
+    for (int k = 0; k < NL; ++k) {
+      const int j = (k / LPP) / NP;
+      wv[k] = make_uint4(0u, tag_in, 0u, tag_in);
+      if (ok[j]) {
+        if constexpr (PE >= 4) {
+          wv[k] = ld_words2_ca(waddr(k));
+        } else {
+          const uint2 w = ld_word_ca(waddr(k));
+          wv[k] = make_uint4(w.x, w.y, 0u, tag_in);
+        }
+      }
+    }
+    uint32_t stale = 0;
+#pragma unroll
+    for (int k = 0; k < NL; ++k)
+      if (!tags_ok(wv[k], tag_in)) stale |= 1u << k;
+    if (stale) {   // rare: a writer's store had not reached L2; re-read those words from L2
+      const uint64_t t0 = globaltimer();
+      for (uint32_t round = 1; stale; ++round) {
+        __nanosleep(32);
+#pragma unroll
+        for (int k = 0; k < NL; ++k)
+          if (stale & (1u << k)) {
+            if constexpr (PE >= 4) {
+              wv[k] = ld_pair2(waddr(k));
+            } else {
+              const uint2 w = ld_pair(waddr(k));
+              wv[k] = make_uint4(w.x, w.y, 0u, tag_in);
+            }
+            if (tags_ok(wv[k], tag_in)) stale &= ~(1u << k);
+          }
+        if (stale && (round & 7) == 0) {
+          if (ld_volatile(p.abort_flag)) break;
+          if (globaltimer() - t0 > p.timeout_ns) { raise_abort(p, 6u << 16); break; }
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NL; ++k) {   // load k covers elements 4k..4k+3 of the thread (2k, 2k+1 for 2-element pieces)
+      if constexpr (PE >= 4) {
+        xv[4 * k] = bf_lo(wv[k].x); xv[4 * k + 1] = bf_hi(wv[k].x);
+        xv[4 * k + 2] = bf_lo(wv[k].z); xv[4 * k + 3] = bf_hi(wv[k].z);
       } else {
-#pragma unroll
-        for (int k = 0; k < PE; ++k) xp[k] = 0.f;
+        xv[2 * k] = bf_lo(wv[k].x); xv[2 * k + 1] = bf_hi(wv[k].x);
       }
     }
   }
+  if (tr && tid == 0) {   // this thread's inputs landed
+    asm volatile("" ::"f"(xv[0]));
+    tr[12] = globaltimer();
+  }
   if (norm) {
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+#pragma unroll
+      for (int c = 0; c < NP; ++c) {
+        float* xp = &xv[(j * NP + c) * PE];
+        if (ok[j]) {   // the gains: read-only, a second (L1 / L2-hit) round trip after the inputs
+          uint32_t gp[PE / 2];
+          ld_bf16_words<PE>(gain + elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c)), gp);
+#pragma unroll
+          for (int k = 0; k < PE; ++k) ss = fmaf(xp[k], xp[k], ss);
+#pragma unroll
+          for (int k = 0; k < PE / 2; ++k) { xp[2 * k] *= bf_lo(gp[k]); xp[2 * k + 1] *= bf_hi(gp[k]); }
+        }
+      }
+    }
     if (rp != 0) ss = 0.f;
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -679,33 +868,43 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
       for (int k = 0; k < PE; ++k) amax = fmaxf(amax, fabsf(xv[c * PE + k]));
       const float q = amax > 0.f ? 32767.f / amax : 0.f;
       asc[c] = amax * (1.f / 32767.f);
-      auto qa = [&](int k) { return __float2int_rn(xv[c * PE + k] * q); };
-      auto pack2 = [](int lo, int hi) { return ((uint32_t)lo & 0xffffu) | ((uint32_t)hi << 16); };
+      // round(x * q) (|x * q| <= 32767, ties to even) without the quarter-rate float-to-int
+      // conversion: the product is rounded to fp32 first (as a conversion of it would be), then
+      // adding 1.5 * 2^23 leaves the integer in the low bits of the sum, whose bit pattern is
+      // 0x4B400000 + round(x * q); its low 16 bits are the int16 in two's complement
+      constexpr float kMagic = 12582912.f;
+      constexpr uint32_t kMagicBits = 0x4B400000u;
+      auto qb = [&](int k) { return __float_as_uint(__fadd_rn(__fmul_rn(xv[c * PE + k], q), kMagic)); };
+      auto pack2 = [](uint32_t lo, uint32_t hi) { return __byte_perm(lo, hi, 0x5410); };   // low halves
       if constexpr (WK == 1) {
 #pragma unroll
-        for (int k = 0; k < PE / 2; ++k) ah[c * PE / 2 + k] = pack2(qa(2 * k), qa(2 * k + 1));
+        for (int k = 0; k < PE / 2; ++k) ah[c * PE / 2 + k] = pack2(qb(2 * k), qb(2 * k + 1));
       } else {
         // a weight word holds elements 8m..8m+7 as nibbles: its low nibbles (elements 0, 2, 4, 6)
         // and high nibbles (1, 3, 5, 7) meet activation words (x0, x2), (x4, x6), (x1, x3), (x5, x7)
-        int sum = 0;
+        uint32_t bsum = 0u;   // sum of the bit patterns: PE * kMagicBits + the sum of the integers
 #pragma unroll
         for (int m = 0; m < PE / 8; ++m) {
-          const int x0 = qa(8 * m), x1 = qa(8 * m + 1), x2 = qa(8 * m + 2), x3 = qa(8 * m + 3);
-          const int x4 = qa(8 * m + 4), x5 = qa(8 * m + 5), x6 = qa(8 * m + 6), x7 = qa(8 * m + 7);
+          const uint32_t x0 = qb(8 * m), x1 = qb(8 * m + 1), x2 = qb(8 * m + 2), x3 = qb(8 * m + 3);
+          const uint32_t x4 = qb(8 * m + 4), x5 = qb(8 * m + 5), x6 = qb(8 * m + 6), x7 = qb(8 * m + 7);
           ah[c * PE / 2 + 4 * m + 0] = pack2(x0, x2);
           ah[c * PE / 2 + 4 * m + 1] = pack2(x4, x6);
           ah[c * PE / 2 + 4 * m + 2] = pack2(x1, x3);
           ah[c * PE / 2 + 4 * m + 3] = pack2(x5, x7);
-          sum += x0 + x1 + x2 + x3 + x4 + x5 + x6 + x7;
+          bsum += x0 + x1 + x2 + x3 + x4 + x5 + x6 + x7;
         }
-        sa[c] = sum;
+        sa[c] = (int)(bsum - (uint32_t)PE * kMagicBits);
       }
     }
   }
 
   if (resid) {   // read back by other threads in the epilogue, behind its barrier
-    if (tid < nrows) s.aux[tid] = rv0;
-    if (tid + kConsumerThreads < nrows) s.aux[tid + kConsumerThreads] = rv1;
+    if (tid < nrows) resid_rows[tid] = rv0;
+    if (tid + kConsumerThreads < nrows) resid_rows[tid + kConsumerThreads] = rv1;
+  }
+  if (tr && tid == 0) {   // stamped once the (quantised) inputs exist
+    if constexpr (IQ) asm volatile("" ::"f"(asc[0]));
+    tr[4] = globaltimer();
   }
 
   // ---- rows, one ring slot at a time ----
@@ -717,6 +916,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
   for (int r0 = 0; r0 < nrows; r0 += g.rs, ++it) {
     const int slot = it % kSlots;
     wait_slot(p, &s.full[slot], (it / kSlots) & 1, (2u << 16) | slot);
+    if (tr && r0 == 0 && tid == 0) tr[5] = globaltimer();
     const int srows = min(g.rs, nrows - r0);
     const uint8_t* sbuf = s.ring + slot * kSlotBytes;
     if (active) {
@@ -798,10 +998,12 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[slot]);
 
-    // ---- epilogue of a finished block of rows ----
+    // ---- epilogue of a finished block of rows: results go out as tagged pairs ----
     const int done = r0 + srows;
     if (done - blk_base == blk_rows || done == nrows) {
+      if (tr && done == nrows && tid == 0) tr[6] = globaltimer();
       bar_compute();
+      if (tr && done == nrows && tid == 0) tr[10] = globaltimer();
       float inv = 1.f;
       if (norm) {
         float t = 0.f;
@@ -810,52 +1012,66 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
         inv = rsqrtf(t / (float)p.d + p.eps);
       }
       const int bs = blk_base, bn = done - blk_base;
+      const uint32_t tag_out = tag_of(ep, l, op == OP_DOWN ? 1 : 0);
       auto rowsum = [&](int rr) {
         float acc = 0.f;
         for (int w = 0; w < g.wpg; ++w) acc += s.part[w * kRowBlock + rr];
         acc *= inv;
         return IQ && sc ? acc * s.scale[bs + rr] : acc;
       };
-      if (op == OP_QKV || op == OP_GU) {
+      if (op == OP_GU) {
+        // four packed rows (gate, up, gate, up) give two SwiGLU outputs: one bf16 pair
+        for (int qd = tid; qd < bn / 4; qd += kConsumerThreads) {
+          const float g0 = rowsum(4 * qd), u0 = rowsum(4 * qd + 1), g1 = rowsum(4 * qd + 2), u1 = rowsum(4 * qd + 3);
+          const float a0 = g0 / (1.f + __expf(-g0)) * u0, a1 = g1 / (1.f + __expf(-g1)) * u1;
+          st_word(p.act + (row0 + bs) / 4 + qd, bf2_word(a0, a1, tag_out));
+        }
+      } else if (op == OP_QKV) {
         for (int pr = tid; pr < bn / 2; pr += kConsumerThreads) {
           const float v0 = rowsum(2 * pr), v1 = rowsum(2 * pr + 1);
           const int gr = row0 + bs + 2 * pr;
-          if (op == OP_GU) {
-            const float silu = v0 / (1.f + __expf(-v0));
-            p.act[gr >> 1] = silu * v1;
-          } else {
+          {
+            // packed rows 2i, 2i + 1 of a head are elements i and i + hd/2 of q, k or v: roped q, roped
+            // k and v go out in packed order, k and v rounded to bf16 as they are cached at pos
             const int hd = p.hd, head = gr / hd, i = (gr % hd) >> 1;
+            float w0 = v0, w1 = v1;
             if (head < p.Hq + p.Hkv) {
-              const float c = s.aux[2 * i], sn = s.aux[2 * i + 1];
-              const float o0 = v0 * c - v1 * sn, o1 = v1 * c + v0 * sn;
-              if (head < p.Hq) {
-                p.q[head * hd + i] = o0;
-                p.q[head * hd + i + hd / 2] = o1;
-              } else {
-                uint16_t* k = p.kcache + (((size_t)l * p.Hkv + (head - p.Hq)) * p.max_seq + p.pos) * hd;
-                k[i] = f2bf(o0);
-                k[i + hd / 2] = f2bf(o1);
-              }
-            } else {
-              uint16_t* vv = p.vcache + (((size_t)l * p.Hkv + (head - p.Hq - p.Hkv)) * p.max_seq + p.pos) * hd;
-              vv[i] = f2bf(v0);
-              vv[i + hd / 2] = f2bf(v1);
+              const float c = resid_rows[2 * i], sn = resid_rows[2 * i + 1];
+              w0 = v0 * c - v1 * sn;
+              w1 = v1 * c + v0 * sn;
             }
+            if (head >= p.Hq) {
+              const bool is_k = head < p.Hq + p.Hkv;
+              uint16_t* kv = (is_k ? p.kcache : p.vcache) +
+                             (((size_t)l * p.Hkv + (head - p.Hq - (is_k ? 0 : p.Hkv))) * p.max_seq + p.pos) * hd;
+              const uint16_t b0 = f2bf(w0), b1 = f2bf(w1);
+              kv[i] = b0;
+              kv[i + hd / 2] = b1;
+              w0 = bf2f(b0);
+              w1 = bf2f(b1);
+            }
+            st_pair2(p.qkv + gr, w0, w1, tag_out);   // gr even: 16-byte aligned
           }
         }
-      } else {
+      } else if (op == OP_LM) {
         for (int rr = tid; rr < bn; rr += kConsumerThreads) {
           const float val = rowsum(rr);
           const int gr = row0 + bs + rr;
-          if (op == OP_LM) {
-            if (p.logits) p.logits[gr] = val;
-            if (val > lm_v || (val == lm_v && gr < lm_i)) { lm_v = val; lm_i = gr; }
-          } else {
-            p.x[gr] = s.aux[bs + rr] + val;
-          }
+          if (p.logits) p.logits[gr] = val;
+          if (val > lm_v || (val == lm_v && gr < lm_i)) { lm_v = val; lm_i = gr; }
+        }
+      } else {
+        // O / down: two rows per thread; the fp32 rows stay this CTA's residual, a bf16 pair goes out
+        for (int pr = tid; pr < bn / 2; pr += kConsumerThreads) {
+          const int gr = row0 + bs + 2 * pr;
+          const float x0 = resid_rows[bs + 2 * pr] + rowsum(2 * pr);
+          const float x1 = resid_rows[bs + 2 * pr + 1] + rowsum(2 * pr + 1);
+          *reinterpret_cast<float2*>(p.xres + gr) = make_float2(x0, x1);
+          st_word(p.x + gr / 2, bf2_word(x0, x1, tag_out));
         }
       }
       bar_compute();
+      if (tr && done == nrows && tid == 0) tr[11] = globaltimer();
       blk_base = done;
     }
   }
@@ -918,43 +1134,54 @@ __device__ __forceinline__ float fast_exp2(float x) {
 __device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : fast_exp2(m - M); }
 
 // Log-sum-exp merge of the C chunk partials (unnormalised o, running max m in log2 units, sum l) of
-// KV head h into attn_out. One thread per (query head, element); a warp holds 32 elements of one
-// query head. Per block of 32 chunks, lane k loads chunk k's (m, l) while every lane loads its own
-// element of all 32 chunks' o, all in one batch (one L2 round trip; a query head's chunks are HD + 2
-// floats apart, so one base address and immediate offsets serve every load); the block max and the
+// KV head h of layer l into the tagged attention output. One thread per (query head, element); a
+// warp holds 32 elements of one query head. Per block of 16 chunks, lane k < 16 loads chunk k's
+// (m, l) pair of pairs while every lane loads its own element of the 16 chunks' o, all in one batch
+// (one L2 round trip: a query head's chunks are hd + 2 pairs apart, so one base address and
+// immediate offsets serve every load; stale tags are re-read together); the block max and the
 // weighted sum of l are warp reductions and each chunk's weight reaches the other lanes by shuffle.
 // Blocks fold into running (M, L, acc) with the usual rescaling, so any C works.
 template <int HD>
-__device__ __noinline__ void merge_head(const Params& p, int h, int C) {
-  constexpr int stride = HD + 2;
+__device__ __noinline__ void merge_head(const Params& p, int h, int C, int l) {
+  constexpr int stride = HD + 2, kBlk = 16;
   const int G = p.Hq / p.Hkv, lane = threadIdx.x & 31;
+  const uint32_t tg = tag_of(p.tag_epoch, l);
   for (int idx = threadIdx.x; idx < G * HD; idx += kConsumerThreads) {   // G * HD: whole warps
     const int g = idx / HD, e = idx % HD;
-    const float* pg = p.attn_part + ((size_t)h * G + g) * p.kv_chunks_max * stride;
+    const uint64_t* pg = p.attn_part + ((size_t)h * G + g) * p.kv_chunks_max * stride;
     float M = -CUDART_INF_F, L = 0.f, acc = 0.f;
-    for (int c0 = 0; c0 < C; c0 += 32) {
-      const int nb = min(32, C - c0);
-      const float* pc = pg + (size_t)c0 * stride;
-      float2 ml = make_float2(-CUDART_INF_F, 0.f);
-      if (lane < nb) ml = __ldcg(reinterpret_cast<const float2*>(pc + lane * stride + HD));
-      float ov[32];
+    for (int c0 = 0; c0 < C; c0 += kBlk) {
+      const int nb = min(kBlk, C - c0);
+      const uint64_t* pc = pg + (size_t)c0 * stride;
+      uint4 ml[1] = {make_uint4(__float_as_uint(-CUDART_INF_F), tg, 0u, tg)};
+      if (lane < nb) ml[0] = ld_pair2(pc + lane * stride + HD);
+      uint2 ov[kBlk];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) ov[k] = k < nb ? __ldcg(pc + k * stride + e) : 0.f;
-      float Mb = fmaxf(M, ml.x);
+      for (int k = 0; k < kBlk; ++k) ov[k] = k < nb ? ld_pair(pc + k * stride + e) : make_uint2(0u, tg);
+      if (!tags_ok(ml[0], tg)) repoll2(p, ml, 1u, tg, [&](int) { return pc + lane * stride + HD; });
+      uint32_t stale = 0;
+#pragma unroll
+      for (int k = 0; k < kBlk; ++k)
+        if (ov[k].y != tg) stale |= 1u << k;
+      if (stale) repoll1(p, ov, stale, tg, [&](int k) { return pc + k * stride + e; });
+      const float mk = __uint_as_float(ml[0].x), lk = __uint_as_float(ml[0].z);
+      float Mb = fmaxf(M, mk);
 #pragma unroll
       for (int o = 16; o; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, o));
-      const float w = exp2_scale(ml.x, Mb);
-      float lsum = ml.y * w;
+      const float w = exp2_scale(mk, Mb);
+      float lsum = lk * w;
 #pragma unroll
       for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
       const float r = exp2_scale(M, Mb);
       L = fmaf(L, r, lsum);
       acc *= r;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) acc = fmaf(ov[k], __shfl_sync(0xffffffffu, w, k), acc);
+      for (int k = 0; k < kBlk; ++k) acc = fmaf(__uint_as_float(ov[k].x), __shfl_sync(0xffffffffu, w, k), acc);
       M = Mb;
     }
-    p.attn_out[(h * G + g) * HD + e] = acc / L;
+    // adjacent elements (lanes 2k, 2k + 1) go out as one bf16 pair
+    const float o = acc / L, o_next = __shfl_down_sync(0xffffffffu, o, 1);
+    if ((e & 1) == 0) st_word(p.attn_out + ((size_t)(h * G + g) * HD + e) / 2, bf2_word(o, o_next, tg));
   }
 }
 
@@ -1000,11 +1227,35 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
   if (p.sync && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
   if (tr && tid == 0) tr[2] = globaltimer();
 
-  // queries of this KV head's group, pre-scaled by log2(e) / sqrt(hd), staged in shared memory
-  // (the GEMV partial-sum region, which attention tasks do not use)
+  // queries of this KV head's group, pre-scaled by log2(e) / sqrt(hd), and this position's key and
+  // value rows (bf16), staged in shared memory (the GEMV partial-sum region, which attention tasks
+  // do not use) in one round trip. The QKV stage publishes them in packed row order: packed row j
+  // of a head is element j / 2 (j even) or hd/2 + j / 2 (j odd).
   const float qs = 1.4426950408889634f * rsqrtf((float)HD);
   float* qsm = s.part;
-  for (int i = tid; i < G * HD; i += kConsumerThreads) qsm[i] = __ldcg(p.q + h * G * HD + i) * qs;
+  uint16_t* kvc = reinterpret_cast<uint16_t*>(s.part + kMaxGroup * 128);   // [HD] k, then [HD] v
+  auto unpack = [](int j) { return (j & 1) ? (j >> 1) + HD / 2 : (j >> 1); };
+  {
+    // up to two tagged pairs of q and (the first 2 * HD threads) one of k or v per thread, all in
+    // one batch (G * HD <= 512)
+    static_assert(kMaxGroup * 128 <= 2 * kConsumerThreads && 2 * 128 <= kConsumerThreads, "q, k, v pairs per thread");
+    const uint32_t tg = tag_of(p.tag_epoch, l);
+    const int ik = tid;
+    const uint64_t* qa = p.qkv + (size_t)h * G * HD;
+    const uint64_t* ka = p.qkv + (size_t)(p.Hq + (ik < HD ? 0 : p.Hkv) + h) * HD + (ik % HD);
+    uint2 v[3] = {make_uint2(0u, tg), make_uint2(0u, tg), make_uint2(0u, tg)};
+    if (tid < G * HD) v[0] = ld_pair(qa + tid);
+    if (tid + kConsumerThreads < G * HD) v[1] = ld_pair(qa + tid + kConsumerThreads);
+    if (ik < 2 * HD) v[2] = ld_pair(ka);
+    const uint32_t stale = (v[0].y != tg ? 1u : 0u) | (v[1].y != tg ? 2u : 0u) | (v[2].y != tg ? 4u : 0u);
+    if (stale) repoll1(p, v, stale, tg, [&](int j) { return j == 2 ? ka : qa + tid + j * kConsumerThreads; });
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int iq = tid + j * kConsumerThreads;
+      if (iq < G * HD) qsm[(iq / HD) * HD + unpack(iq % HD)] = __uint_as_float(v[j].x) * qs;
+    }
+    if (ik < 2 * HD) kvc[(ik < HD ? 0 : HD) + unpack(ik % HD)] = f2bf(__uint_as_float(v[2].x));
+  }
   bar_compute();
 
   float m[HW], ls[HW], o[HW][8];
@@ -1027,7 +1278,6 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
     }
   }
 
-  const size_t head_off = ((size_t)l * p.Hkv + h) * p.max_seq;
   for (int blk = cb; blk < ce; blk += NPS, ++it) {
     const int slot = it % kSlots;
     wait_slot(p, &s.full[slot], (it / kSlots) & 1, (2u << 16) | slot);
@@ -1035,13 +1285,12 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
     uint8_t* kb = s.ring + slot * kSlotBytes;
     uint8_t* vb = kb + kSlotBytes / 2;
     if (p.pos >= blk && p.pos < blk + n) {
-      // this step's own key/value row: written by the QKV stage, read with plain loads
+      // this step's own key/value row (not copied: the QKV stage writes it in this launch) from the
+      // staged copy; the proxy fence orders these generic writes before the slot's next bulk copy
       const int j = p.pos - blk;
       if (tid < HD / 4) {
-        const uint2* ks = reinterpret_cast<const uint2*>(p.kcache + (head_off + p.pos) * HD);
-        const uint2* vs = reinterpret_cast<const uint2*>(p.vcache + (head_off + p.pos) * HD);
-        reinterpret_cast<uint2*>(kb + (size_t)j * HD * 2)[tid] = __ldcg(ks + tid);
-        reinterpret_cast<uint2*>(vb + (size_t)j * HD * 2)[tid] = __ldcg(vs + tid);
+        reinterpret_cast<uint2*>(kb + (size_t)j * HD * 2)[tid] = reinterpret_cast<const uint2*>(kvc)[tid];
+        reinterpret_cast<uint2*>(vb + (size_t)j * HD * 2)[tid] = reinterpret_cast<const uint2*>(kvc + HD)[tid];
         fence_proxy_async_smem();
       }
       bar_compute();
@@ -1113,6 +1362,7 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
     if (lane == 0) mbar_arrive(&s.empty[slot]);
   }
 
+  if (tr && tid == 0) tr[4] = globaltimer();
   // merge the sub-warps of this warp (lanes with the same piece)
 #pragma unroll
   for (int g = 0; g < HW; ++g) {
@@ -1180,29 +1430,28 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
       L = fmaf(ew[HD + 1], wt, L);
       acc = fmaf(ew[e], wt, acc);
     }
-    float* dg = p.attn_part + (((size_t)h * G + g) * p.kv_chunks_max + c) * stride;
-    dg[e] = acc;
-    if (e == 0) { dg[HD] = M; dg[HD + 1] = L; }
+    uint64_t* dg = p.attn_part + (((size_t)h * G + g) * p.kv_chunks_max + c) * stride;
+    const uint32_t tg = tag_of(p.tag_epoch, l);
+    st_pair(dg + e, acc, tg);
+    if (e == 0) st_pair2(dg + HD, M, L, tg);   // (hd + 2) even: 16-byte aligned
   }
+  if (tr && tid == 0) tr[5] = globaltimer();
   if (!p.sync) return it;
-  // ticket: the last chunk of this head to finish merges all of them and signals. The ticket is an
-  // acquire-release atomic: it publishes this CTA's partial (made visible to thread 0 by the
-  // barrier) and, for the last arrival, acquires every earlier chunk's.
+  // ticket: the last chunk of this head to arrive merges all of them and signals. A relaxed atomic:
+  // the merge checks the tags of every partial it reads.
   bar_compute();
   uint32_t* ticket = p.attn_ticket + l * p.Hkv + h;
-  if (tid == 0) {
-    uint32_t old;
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
-    s.misc->flag = (old == (uint32_t)(C - 1));
-  }
+  if (tid == 0) s.misc->flag = (atom_relaxed_add(ticket, 1u) == (uint32_t)(C - 1));
   bar_compute();
+  if (tr && tid == 0) tr[6] = globaltimer();
   if (s.misc->flag) {
-    merge_head<HD>(p, h, C);
+    merge_head<HD>(p, h, C, l);
     bar_compute();
     if (tid == 0) {
       *ticket = 0u;
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.ctr + t.sig_ctr) : "memory");
+      red_relaxed_add(p.ctr + t.sig_ctr, 1u);
     }
+    if (tr && tid == 0) tr[7] = globaltimer();
   }
   bar_compute();
   return it;
@@ -1216,9 +1465,13 @@ __device__ __noinline__ void grid_argmax(const Params& p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float bv = -CUDART_INF_F;
   int bi = 0x7fffffff;
+  const uint32_t tg = tag_of(p.tag_epoch, p.L);
   for (int b = threadIdx.x; b < p.grid; b += kConsumerThreads) {
-    const float v = __ldcg(p.am_val + b);
-    const int i = __ldcg(p.am_idx + b);
+    // {max, index} as two tagged pairs: re-read until both tags are this launch's (bounded)
+    uint4 e[1] = {ld_pair2(p.am + 2 * b)};
+    if (!tags_ok(e[0], tg)) repoll2(p, e, 1u, tg, [&](int) { return p.am + 2 * b; });
+    const float v = __uint_as_float(e[0].x);
+    const int i = (int)e[0].z;
     if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
   }
 #pragma unroll
@@ -1259,14 +1512,10 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
   }
   bar_compute();
   const int token = s.misc->token;
-  if (p.init_x) {
-    const int r0 = p.o_rows[2 * blockIdx.x], n = p.o_rows[2 * blockIdx.x + 1];
-    for (int r = tid; r < n; r += kConsumerThreads) p.x[r0 + r] = bf2f(p.embed[(size_t)token * p.d + r0 + r]);
-  }
   uint32_t it = 0;
   for (int ti = 0; ti < nt; ++ti) {
     const Task t = tasks[ti];
-    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_tasks_per_cta + ti) * 4 : nullptr;
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_tasks_per_cta + ti) * AMK_TRACE_WORDS : nullptr;
     if (tr && tid == 0) {
       tr[0] = ((unsigned long long)t.op << 32) | (unsigned long long)t.layer << 16 | (unsigned)ti;
       tr[1] = tr[2] = globaltimer();
@@ -1310,17 +1559,15 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
       }
       if (t.op == OP_LM) {
         if (t.flags & kLastOfStage) {
-          if (tid == 0) { p.am_val[blockIdx.x] = s.misc->lm_v; p.am_idx[blockIdx.x] = s.misc->lm_i; }
+          // this CTA's maximum as one tagged 16-byte store; the last CTA to take the ticket reduces
+          // them all, re-reading any entry whose tags are not this launch's yet (no fence needed)
+          if (tid == 0)
+            st_pair2(p.am + 2 * blockIdx.x, s.misc->lm_v, __int_as_float(s.misc->lm_i), tag_of(p.tag_epoch, p.L));
           if (p.sync) {
             bar_compute();
-            if (tid == 0) {
-              __threadfence();
-              const uint32_t old = atomicAdd(p.am_ticket, 1u);
-              s.misc->flag = (old == (uint32_t)(p.grid - 1));
-            }
+            if (tid == 0) s.misc->flag = (atom_relaxed_add(p.am_ticket, 1u) == (uint32_t)(p.grid - 1));
             bar_compute();
             if (s.misc->flag) {
-              __threadfence();
               grid_argmax(p);
               if (tid == 0) *p.am_ticket = 0u;
             }
@@ -1330,13 +1577,14 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
         bar_compute();
         signal_counter(p, t.sig_ctr);
       }
+      if (tr && tid == 0) tr[7] = globaltimer();
     } else if (t.op == OP_ATTN) {
       if (p.hd == 64) it = attn_task<64>(p, t, it, tr);
       else it = attn_task<128>(p, t, it, tr);
     } else if (t.op == OP_MERGE) {
       const int C = attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max);
-      if (p.hd == 64) merge_head<64>(p, t.a, C);
-      else merge_head<128>(p, t.a, C);
+      if (p.hd == 64) merge_head<64>(p, t.a, C, t.layer);
+      else merge_head<128>(p, t.a, C, t.layer);
     } else if (t.op == OP_ARGMAX) {
       grid_argmax(p);
     }

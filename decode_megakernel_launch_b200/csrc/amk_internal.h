@@ -20,8 +20,13 @@
 namespace amk {
 
 // ---- CTA shape and shared-memory budget ------------------------------------------------------
-constexpr int kConsumerWarps   = 16;
-constexpr int kConsumerThreads = kConsumerWarps * 32;      // 512 compute threads
+// Compute warps (a compile-time knob). With the producer, 17 warps put 5 on one SM sub-partition,
+// which caps every thread at 96 registers; 15 + 1 would leave 128.
+#ifndef AMK_CONSUMER_WARPS
+#define AMK_CONSUMER_WARPS 16
+#endif
+constexpr int kConsumerWarps   = AMK_CONSUMER_WARPS;
+constexpr int kConsumerThreads = kConsumerWarps * 32;      // compute threads
 constexpr int kThreads         = kConsumerThreads + 32;    // + 1 producer (bulk-copy) warp
 // Ring geometry (compile-time; -DAMK_SLOT_BYTES / -DAMK_SLOTS / -DAMK_INFLIGHT override it).
 // kInflight bounds the copies the producer keeps outstanding: every other global access of the SM
@@ -58,7 +63,7 @@ constexpr unsigned kStallNs = AMK_PF_STALL_NS;
 static_assert(kInflight >= 1 && kInflight <= kSlots, "ring in-flight bound");
 static_assert(kSlotBytes % 256 == 0 && kSlotBytes >= 32768, "ring slot holds a 32 KB weight row");
 constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block
-constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV task (scale cache)
+constexpr int kMaxTaskRows     = kConsumerThreads * 2 >= 1024 ? 1024 : kConsumerThreads * 2;   // rows of one GEMV task
 // Rows per register batch of the GEMV inner loop for 64- and 32-byte groups (the transposed
 // butterfly reduces 2 or 4 rows at once).
 #ifndef AMK_NB64
@@ -70,6 +75,14 @@ constexpr int kMaxTaskRows     = 1024;                     // rows of one GEMV t
 // Largest int4 group (bytes of nibbles per thread per row): 16 B = 32 elements, 32 B = 64.
 #ifndef AMK_I4_MAX_GB
 #define AMK_I4_MAX_GB 16
+#endif
+// The hot GEMV instances (int8 with 32-byte groups, int4 with 16-byte groups, one group per thread)
+// inlined into the kernel's task loop (1) or called (0).
+#ifndef AMK_INLINE_HOT
+#define AMK_INLINE_HOT 1
+#endif
+#ifndef AMK_INLINE_HOT4
+#define AMK_INLINE_HOT4 1
 #endif
 // int4 high nibbles: masked in place and met with an unsigned-byte dp2a (1) or shifted down (0).
 #ifndef AMK_I4_NOSHIFT
@@ -86,6 +99,22 @@ constexpr int kTaskCacheBytes  = kTaskCache * 32;
 constexpr int kSmemBytes       = kRingBytes + kPartBytes + kAuxBytes + kScaleBytes + kMiscBytes + kTaskCacheBytes;
 static_assert(kSmemBytes <= 227 * 1024, "dynamic shared memory of one CTA");
 static_assert(kAuxBytes >= kMaxTaskRows * 4 && kAuxBytes >= 128 * 4, "aux holds a GEMV task's residual rows or a RoPE row");
+
+// ---- tagged activations ----------------------------------------------------------------------
+// Every vector one CTA hands to others travels in 64-bit tagged words, each one aligned 8-byte
+// element of the store that writes it and of the load that reads it, so a reader that sees the tag
+// sees the payload: the high word is the tag, the low word either two bf16 values (the GEMV inputs:
+// x after O and after down, the merged attention, the SwiGLU output; the 16-bit activations of
+// W8A16) or one fp32 value (the packed q / k / v rows, the attention partials, the LM-head maxima).
+// A reader accepts a word only when its tag is the one it expects and re-reads the others, so the
+// writer needs no release fence (under the full weight stream a gpu-scope fence costs several
+// microseconds: it waits on the SM's in-flight weight copies); the stage counters, bumped with
+// relaxed reductions, only tell readers of a wide vector when to start reading it. The residual
+// stream itself stays fp32: each CTA keeps its own rows of x (O and down split rows the same way).
+// The tag names the launch, the layer and (for x) the version: tag = epoch * 2048 + 2 * layer + k,
+// k = 0 for x after O and for every other vector, 1 for x after down.
+AMK_HD inline uint32_t tag_of(uint32_t epoch, int layer, int k = 0) { return epoch * 2048u + 2u * (uint32_t)layer + (uint32_t)k; }
+constexpr int kMaxLayers = 1023;   // 2 * layer + 1 < 2048, the LM head's entries use layer = n_layers
 
 // ---- tasks -----------------------------------------------------------------------------------
 enum Op : uint16_t {
@@ -168,13 +197,15 @@ struct Params {
   uint16_t* vcache;
   const float* rope;           // interleaved (cos, sin) [max_seq][hd/2][2]
   // scratch (device)
-  float* x;                    // residual stream [d]
-  float* q;                    // roped queries [Hq*hd]
-  float* attn_out;             // merged attention [Hq*hd]
-  float* act;                  // SwiGLU output [ffn]
-  float* attn_part;            // [Hkv][G][kv_chunks_max][hd + 2]: o, then m and l of each chunk
-  float* am_val;               // per-CTA LM maxima [grid]
-  int*   am_idx;
+  // tagged words (see tag_of)
+  uint64_t* x;                 // x as bf16 pairs [d / 2] (after O, then after down)
+  float* xres;                 // x in fp32 [d]: each CTA reads back only the rows it wrote
+  uint64_t* qkv;               // QKV outputs in packed row order [(Hq + 2 Hkv) hd], fp32: roped q, roped k
+                               //   and v rounded to bf16 (this position's keys and values, as cached)
+  uint64_t* attn_out;          // merged attention as bf16 pairs [Hq * hd / 2]
+  uint64_t* act;               // SwiGLU output as bf16 pairs [ffn / 2]
+  uint64_t* attn_part;         // [Hkv][G][kv_chunks_max][hd + 2], fp32: o, then m and l of each chunk
+  uint64_t* am;                // [grid][2] LM-head maximum and its index
   uint32_t* ctr;               // [L * CTR_PER_LAYER]
   uint32_t* attn_ticket;       // [L * Hkv]
   uint32_t* am_ticket;         // [1]
@@ -190,14 +221,13 @@ struct Params {
   int kv_chunks_max;
   unsigned long long timeout_ns;
   // per launch
-  uint32_t epoch;
+  uint32_t epoch;              // counter targets are epoch * producers
+  uint32_t tag_epoch;          // tags of this launch's vectors (tag_of)
   int token;                   // >= 0, or -1 to read *next_token
   int pos;
   float* logits;               // may be null
   int*   next_token;
   int sync;                    // 1 = persistent megakernel (waits/signals), 0 = op-per-kernel
-  int init_x;                  // this launch writes x = E[token] for its O rows first
-  const int* o_rows;           // [grid][2] (row0, nrows) of each CTA's O tasks (for init_x)
 };
 
 // ---- shared host/device helpers ----------------------------------------------------------------

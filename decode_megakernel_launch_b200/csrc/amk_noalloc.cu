@@ -54,6 +54,7 @@ struct DeviceSlot {
   std::vector<const void*> ptrs;   // weight / cache pointers the uploaded LayerPtrs came from
   Params base_params{};
   size_t zero_off = 0, zero_bytes = 0;
+  uint32_t tag_epoch = 0;          // tag epoch of the last call
 };
 
 std::mutex g_mu;
@@ -132,16 +133,16 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
     auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
     const size_t o_tasks = take(pl.tasks.size() * sizeof(Task));
     const size_t o_off = take(pl.off.size() * sizeof(int));
-    const size_t o_orows = take(pl.o_rows.size() * sizeof(int));
     const size_t o_layers = take((size_t)L * sizeof(LayerPtrs));
     const size_t o_rope = take((size_t)d.max_seq * half * 2 * sizeof(float));
-    const size_t o_x = take((size_t)d.d_model * 4);
-    const size_t o_q = take((size_t)d.n_q_heads * d.head_dim * 4);
-    const size_t o_ao = take((size_t)d.n_q_heads * d.head_dim * 4);
-    const size_t o_act = take((size_t)d.ffn * 4);
-    const size_t o_part = take((size_t)d.n_kv_heads * pl.kv_chunks_max * G * (d.head_dim + 2) * 4);
-    const size_t o_amv = take((size_t)grid * 4);
-    const size_t o_ami = take((size_t)grid * 4);
+    const size_t tagged_begin = off;                      // tagged vectors: zeroed on every reload
+    const size_t o_x = take((size_t)d.d_model / 2 * 8);
+    const size_t o_xres = take((size_t)d.d_model * 4);
+    const size_t o_qkv = take((size_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * 8);
+    const size_t o_ao = take((size_t)d.n_q_heads * d.head_dim / 2 * 8);
+    const size_t o_act = take((size_t)d.ffn / 2 * 8);
+    const size_t o_part = take((size_t)d.n_kv_heads * pl.kv_chunks_max * G * (d.head_dim + 2) * 8);
+    const size_t o_am = take((size_t)grid * 16);
     const size_t zero_begin = off;                        // everything below must start at zero
     const size_t o_ctr = take((size_t)pl.n_counters * 4);
     const size_t o_tix = take((size_t)L * d.n_kv_heads * 4);
@@ -174,9 +175,11 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
     };
     if (!put(o_tasks, pl.tasks.data(), pl.tasks.size() * sizeof(Task)) ||
         !put(o_off, pl.off.data(), pl.off.size() * sizeof(int)) ||
-        !put(o_orows, pl.o_rows.data(), pl.o_rows.size() * sizeof(int)) ||
         !put(o_layers, lp.data(), lp.size() * sizeof(LayerPtrs)) || !put(o_rope, rope.data(), rope.size() * 4))
       return AMK_ERR_CUDA;
+    // tag 0 never matches (tag epochs start at 1): no value left by another model passes a check
+    if (cudaMemsetAsync(B + tagged_begin, 0, zero_begin - tagged_begin, st) != cudaSuccess) return AMK_ERR_CUDA;
+    S.tag_epoch = 0;
 
     Params& p = S.base_params;
     p = Params{};
@@ -191,13 +194,13 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
     p.kcache = static_cast<uint16_t*>(w->k_cache);
     p.vcache = static_cast<uint16_t*>(w->v_cache);
     p.rope = reinterpret_cast<const float*>(B + o_rope);
-    p.x = reinterpret_cast<float*>(B + o_x);
-    p.q = reinterpret_cast<float*>(B + o_q);
-    p.attn_out = reinterpret_cast<float*>(B + o_ao);
-    p.act = reinterpret_cast<float*>(B + o_act);
-    p.attn_part = reinterpret_cast<float*>(B + o_part);
-    p.am_val = reinterpret_cast<float*>(B + o_amv);
-    p.am_idx = reinterpret_cast<int*>(B + o_ami);
+    p.x = reinterpret_cast<uint64_t*>(B + o_x);
+    p.xres = reinterpret_cast<float*>(B + o_xres);
+    p.qkv = reinterpret_cast<uint64_t*>(B + o_qkv);
+    p.attn_out = reinterpret_cast<uint64_t*>(B + o_ao);
+    p.act = reinterpret_cast<uint64_t*>(B + o_act);
+    p.attn_part = reinterpret_cast<uint64_t*>(B + o_part);
+    p.am = reinterpret_cast<uint64_t*>(B + o_am);
     p.ctr = reinterpret_cast<uint32_t*>(B + o_ctr);
     p.attn_ticket = reinterpret_cast<uint32_t*>(B + o_tix);
     p.am_ticket = reinterpret_cast<uint32_t*>(B + o_amt);
@@ -207,7 +210,6 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
     p.max_tasks_per_cta = 0;
     p.tasks = reinterpret_cast<const Task*>(B + o_tasks);
     p.task_off = reinterpret_cast<const int*>(B + o_off);
-    p.o_rows = reinterpret_cast<const int*>(B + o_orows);
     for (int i = 0; i < 5; ++i) p.geom[i] = pl.geom[i];
     p.kv_block = 64;
     p.kv_chunks_max = pl.kv_chunks_max;
@@ -221,13 +223,16 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
 
   // ---- per call: zero the counters / tickets / status, then one persistent launch ----
   if (cudaMemsetAsync(S.base + S.zero_off, 0, S.zero_bytes, st) != cudaSuccess) return AMK_ERR_CUDA;
+  // counters restart from zero each call, so their targets use epoch 1; the tags use a running
+  // epoch, so no value left in the array by an earlier call passes a check
   Params p = S.base_params;
   p.epoch = 1;
+  S.tag_epoch = S.tag_epoch + 1 == 0 ? 1 : S.tag_epoch + 1;
+  p.tag_epoch = S.tag_epoch;
   p.token = token_id;
   p.pos = pos;
   p.logits = logits_out;
   p.next_token = next_token_out;
   p.sync = 1;
-  p.init_x = 1;
   return launch_decode(p, st, true) == cudaSuccess ? AMK_OK : AMK_ERR_CUDA;
 }

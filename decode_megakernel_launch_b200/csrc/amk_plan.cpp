@@ -83,9 +83,13 @@ bool make_geom(int K, int wk, GemvGeom* g) {
     double score = bal * eff[i];
     if (score > best + 1e-9) {
       best = score;
+      // rows per slot: a power of two below 8, else a multiple of 8, so every 128-row epilogue block
+      // (rs * floor(128 / rs) rows) is a multiple of 8 rows: its results go out in bf16 pairs of
+      // rows (SwiGLU: of two packed row pairs)
       int rs = kSlotBytes / rb;
       if (rs > 64) rs = 64;
-      if (rs > 1 && (rs & 1)) rs -= 1;
+      if (rs >= 8) rs &= ~7;
+      else rs = rs >= 4 ? 4 : rs >= 2 ? 2 : 1;
       *g = GemvGeom{K, rb, gb, W, wpg, nr, rp, rs};
       found = true;
     }
@@ -96,7 +100,7 @@ bool make_geom(int K, int wk, GemvGeom* g) {
 int check_dims(const amk_dims& d, std::string* msg) {
   auto bad = [&](const char* m) { *msg = m; return AMK_ERR_UNSUPPORTED; };
   if (d.n_layers < 1 || d.d_model < 1 || d.n_q_heads < 1 || d.n_kv_heads < 1 || d.ffn < 1 || d.vocab < 1 ||
-      d.max_seq < 1 || d.n_layers > 65535) {
+      d.max_seq < 1 || d.n_layers > kMaxLayers) {
     *msg = "dims must be positive";
     return AMK_ERR_INVALID_ARG;
   }
@@ -129,7 +133,8 @@ int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::s
   int L = d.n_layers, hd = d.head_dim, Hkv = d.n_kv_heads;
   // attention chunks per KV head; the (head, chunk) tasks go round-robin over the CTAs, so a grid
   // smaller than Hkv gives some CTAs several heads
-  int cmax = kv_chunks_max > 0 ? kv_chunks_max : grid / Hkv;
+  // at most 16 chunks per KV head by default: the merge then gathers them in one round trip
+  int cmax = kv_chunks_max > 0 ? kv_chunks_max : std::min(grid / Hkv, 16);
   if (cmax < 1) cmax = 1;
   p.kv_chunks_max = cmax;
   p.n_counters = L * CTR_PER_LAYER;
@@ -140,11 +145,13 @@ int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::s
   make_geom(d.ffn, wk, &p.geom[3]);                               // DOWN:K = ffn
   make_geom(d.d_model, d.tied_head ? AMK_W_BF16 : wk, &p.geom[4]);  // LM: its own dtype, or the bf16 table
 
+  // results go out in pairs: QKV row pairs (RoPE), O / down rows two by two (one bf16 pair each),
+  // gate/up four packed rows at a time (two SwiGLU outputs, one bf16 pair)
   int qkv_rows = (d.n_q_heads + 2 * Hkv) * hd;
   auto s_qkv = split_rows(qkv_rows, 2, grid);
-  auto s_o = split_rows(d.d_model, 1, grid);
-  auto s_gu = split_rows(2 * d.ffn, 2, grid);
-  auto s_dn = split_rows(d.d_model, 1, grid);
+  auto s_o = split_rows(d.d_model, 2, grid);
+  auto s_gu = split_rows(2 * d.ffn, 4, grid);
+  auto s_dn = split_rows(d.d_model, 2, grid);
   auto s_lm = split_rows(d.vocab, 1, grid);
   // remainder rows of an odd split go to the last CTA
   auto fix_tail = [&](std::vector<Split>& s, int n) {
@@ -155,8 +162,6 @@ int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::s
   fix_tail(s_dn, d.d_model);
   fix_tail(s_lm, d.vocab);
 
-  p.o_rows.resize(2 * grid);
-  for (int b = 0; b < grid; ++b) { p.o_rows[2 * b] = s_o[b].row0; p.o_rows[2 * b + 1] = s_o[b].nrows; }
 
   // Appends the tasks of one GEMV stage for CTA b: rows split into pieces of <= kMaxTaskRows
   // (even sizes for pair-wise epilogues); the first piece waits, the last signals. A CTA without
@@ -351,9 +356,11 @@ int check_plan(const amk_dims& d, const Plan& p, std::string* msg) {
     }
     if (r != need(kv.first.first)) return fail(fmt("stage %ld layer %ld covers %ld rows", kv.first.first, kv.first.second, r));
   }
-  // pair-wise epilogues need even row starts and counts
-  for (const Task& t : p.tasks)
-    if ((t.op == OP_QKV || t.op == OP_GU) && ((t.a | t.b) & 1)) return fail("QKV / gate-up task split inside a row pair");
+  // pair-wise epilogues: QKV, O and down rows in pairs, gate/up rows in fours
+  for (const Task& t : p.tasks) {
+    const int unit = t.op == OP_GU ? 4 : (t.op == OP_QKV || t.op == OP_O || t.op == OP_DOWN) ? 2 : 1;
+    if ((t.a % unit) || (t.b % unit)) return fail(fmt("stage %ld: task rows %ld + %ld split a row pair", t.op, t.a, t.b));
+  }
   *msg = "ok";
   return AMK_OK;
 }

@@ -21,7 +21,6 @@ struct Plan {
   std::vector<Task> tasks;        // persistent kernel: all CTAs' lists back to back
   std::vector<int> off;           // [grid + 1]
   std::vector<StageList> stages;  // ablation launches in order
-  std::vector<int> o_rows;        // [grid * 2]: (row0, nrows) of each CTA's O rows
 };
 
 // Geometry of one GEMV with rows of K elements of weight dtype `wk` (AMK_W_*); false if unsupported.

@@ -148,11 +148,12 @@ class DeviceModel:
 
     def trace(self, max_records: int = 1 << 20):
         import numpy as np
-        buf = (C.c_uint64 * (4 * max_records))()
+        w = amk.AMK_TRACE_WORDS
+        buf = (C.c_uint64 * (w * max_records))()
         n = amk.amk_trace_read(self.handle, buf, max_records)
         if n < 0:
             raise amk.AmkError("amk_trace_read", n)
-        return np.frombuffer(buf, dtype=np.uint64, count=4 * n).reshape(n, 4).copy()
+        return np.frombuffer(buf, dtype=np.uint64, count=w * n).reshape(n, w).copy()
 
     def close(self) -> None:
         if self.handle is not None:

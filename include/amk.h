@@ -100,7 +100,7 @@ typedef struct amk_weights {
 typedef struct amk_options {
   int grid;              /* persistent CTAs; 0 = one per SM                                    */
   int kv_block;          /* minimum positions per attention chunk; 0 = 64                      */
-  int max_kv_chunks;     /* cap on attention chunks per KV head; 0 = grid / Hkv                */
+  int max_kv_chunks;     /* cap on attention chunks per KV head; 0 = min(grid / Hkv, 16)       */
   int timeout_ms;        /* bound on every device wait; 0 = 2000 ms                            */
   int trace;             /* 1: record per-task timestamps (see amk_trace_read)                 */
   int test_drop_signal;  /* TEST ONLY: 1 + index of a counter signal the planner omits, so the
@@ -230,11 +230,21 @@ int amk_plan_check(const amk_dims* dims, int grid, int mutation, char* msg, int 
 
 /* ---- tracing --------------------------------------------------------------------------------- */
 
-/* With options.trace = 1, every CTA records (task, wait-start, wait-end, done) %globaltimer
- * stamps (ns) of the last step. Copies up to `max_records` records of 4 uint64 each into the host
- * buffer `out` (synchronizes the device) and returns how many were written, or a negative code.
- * Record r of CTA b is at index b * (max tasks per CTA) + r; unused records are zero. The task word
- * holds (op << 32) | (layer << 16) | (index of the task in its CTA's list), op one of: */
+/* With options.trace = 1, every CTA records AMK_TRACE_WORDS uint64 per task of the last step:
+ *   [0] task word, [1] start, [2] inputs may be read (its counter seen), [3] done, and
+ *   %globaltimer stamps (ns) of its phases:
+ *   GEMV:      [4] inputs loaded and quantised, [5] first ring slot landed, [6] thread 0's last row
+ *              computed, [10] every warp's last row computed, [11] last result block's bulk store
+ *              issued, [7] signal issued (after that store completed);
+ *   attention: [4] KV chunk done, [5] partial issued, [6] ticket taken, [7] head merged and signalled
+ *              (0 unless this chunk merged the head);
+ *   producer:  [8] the task's first ring item issued, [9] its last item issued;
+ *   GEMV inputs: [12] thread 0's input words landed.
+ * Copies up to `max_records` records into the host buffer `out` (synchronizes the device) and
+ * returns how many were written, or a negative code. Record r of CTA b is at index
+ * b * (max tasks per CTA) + r; unused records and stamps are zero. The task word holds
+ * (op << 32) | (layer << 16) | (index of the task in its CTA's list), op one of: */
+#define AMK_TRACE_WORDS 16
 #define AMK_OP_QKV  1   /* RMSNorm -> QKV GEMV -> RoPE -> K/V append                         */
 #define AMK_OP_ATTN 2   /* attention of one KV head over one KV chunk (+ the head's merge)    */
 #define AMK_OP_O    3   /* O GEMV + residual                                                  */
