@@ -28,11 +28,16 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 decode tokens/s (W8A16) and achieved HBM GB/s vs B200 peak"
-DTYPE_TEXT = {"int8": "w8a16: int8 weights (bf16 row scales) x int16 activations quantised per 16 elements "
-                      "(fp32 scale), exact int32 dot per 16 elements, fp32 accumulate",
-              "int4": "w4a16: int4 weights (bf16 row scales) x int16 activations quantised per 32 elements "
-                      "(fp32 scale), exact int32 dot per 32 elements, fp32 accumulate",
-              "bf16": "bf16 weights x fp32 activations, fp32 accumulate"}
+DTYPE_TEXT = {"int8": "w8a16: int8 weights (bf16 row scales) x bf16 activations, quantised in the GEMV to int16 "
+                      "per 16 elements (fp32 scale), exact int32 dot per 16 elements, fp32 accumulate; fp32 residual",
+              "int4": "w4a16: int4 weights (bf16 row scales) x bf16 activations, quantised in the GEMV to int16 "
+                      "per 32 elements (fp32 scale), exact int32 dot per 32 elements, fp32 accumulate; fp32 residual",
+              "bf16": "bf16 weights x bf16 activations, fp32 accumulate; fp32 residual"}
+# Every named shape, measured in the same run after the headline workload (bounded windows).
+CONFIG_SET = [("smollm135m", {}), ("llama1b", {}), ("llama1b", {"weight_dtype": "bf16"}),
+              ("llama8b", {"weight_dtype": "bf16"}), ("llama8b_int4", {}), ("llama1b_long4k", {}),
+              ("llama1b_long16k", {}), ("llama1b_long32k", {})]
+L2_BYTES = 126e6
 
 
 def metric_for(cfg) -> str:
@@ -186,6 +191,72 @@ def run_reference(args, cfg, rank, world):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
+
+
+def measure_config(cfg, peak, steps=32, warmup=8, ablation_steps=4):
+    """One named shape in a bounded window: tokens/s, per-token latency p50/p99, algorithmic bytes, GB/s
+    and its fraction of the HBM peak, the op-per-kernel ablation, and the critical path per op of one
+    traced step (for the long-context shapes also the attention share of bytes and of time)."""
+    import torch
+    from decode_megakernel_launch_b200 import synth
+    from decode_megakernel_launch_b200.runtime import DeviceModel, stage_breakdown
+    t0 = time.time()
+    model = DeviceModel(cfg)
+    if cfg.prompt_len:
+        for i, t in enumerate(synth.prompt_ids(cfg)):
+            model.step(t, i)
+    start = cfg.prefill_len + cfg.prompt_len
+    span = max(1, cfg.decode_steps)
+    pos_of = lambda k: start + k % span
+    model.next_token.fill_(1)
+    for k in range(warmup):
+        model.step(-1 if k else 1, pos_of(k))
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record()
+        model.step(-1, pos_of(warmup + k))
+        ev[k][1].record()
+    torch.cuda.synchronize()
+    per = sorted(a.elapsed_time(b) for a, b in ev)
+    rc, detail = model.status()
+    if rc != 0:
+        raise RuntimeError(f"{cfg.name}: device status {rc} detail {detail:#x}")
+    ms = sum(per) / len(per)
+    by = sum(model.step_bytes(pos_of(warmup + k)) for k in range(steps)) / steps
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for k in range(ablation_steps):
+        model.step(-1, pos_of(k), unfused=True)
+    a1.record()
+    torch.cuda.synchronize()
+    out = {"workload": _workload_name(cfg), "tokens_per_s": 1000.0 / ms, "ms_per_token": ms, "p50_ms": per[len(per) // 2],
+           "p99_ms": per[min(len(per) - 1, int(0.99 * len(per)))], "bytes_per_step": by,
+           "achieved_gbs": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / peak,
+           "unfused_ms_per_token": a0.elapsed_time(a1) / ablation_steps, "steps": steps}
+    if by < 2 * L2_BYTES:
+        out["l2_note"] = (f"{by / 1e6:.0f} MB per token against a {L2_BYTES / 1e6:.0f} MB L2: weights stay partly "
+                          "L2-resident between steps, so GB/s may exceed what HBM alone gives")
+    try:
+        model.close()
+        model._create(dict(trace=1))
+        model.next_token.fill_(1)
+        for k in range(3):
+            model.step(-1 if k else 1, pos_of(k))
+        bd = stage_breakdown(model.trace())
+        out["stage_us"] = {k: round(v, 1) for k, v in bd["us"].items()}
+        out["span_us"] = round(bd["span_us"], 1)
+        if cfg.prefill_len >= 4096:
+            kv = 2.0 * cfg.n_layers * cfg.n_kv_heads * (pos_of(2) + 1) * cfg.head_dim * 2
+            out["attention_share"] = {"bytes": kv / model.step_bytes(pos_of(2)),
+                                      "time": bd["us"].get("attn", 0.0) / max(bd["span_us"], 1e-9)}
+    except Exception as e:  # diagnostics only
+        out["stage_us"] = f"unavailable: {type(e).__name__}"
+    model.close()
+    del model
+    torch.cuda.empty_cache()
+    out["seconds"] = round(time.time() - t0, 1)
+    return out
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -353,6 +424,23 @@ def run_gpu(args, cfg, rank, world, local_rank):
                "seconds": round(secs, 1)}
 
     traffic = _dram_traffic(cfg.name, avg_bytes)
+    # the headline model's device memory goes before the other shapes and the comparator load theirs
+    model.close()
+    del model
+    import gc
+    gc.collect()
+    torch.cuda.empty_cache()
+    configs = None
+    if rank == 0 and world == 1 and not args.no_configs:
+        from decode_megakernel_launch_b200 import synth as _synth
+        configs = {}
+        for name, over in CONFIG_SET:
+            c = _synth.preset(name, **over)
+            key = f"{name}_{c.weight_dtype}" if over else name
+            try:
+                configs[key] = measure_config(c, peak)
+            except Exception as e:  # one shape failing must not hide the headline
+                configs[key] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     comparator = None
     if world == 1 and not args.no_comparator:
         try:
@@ -384,10 +472,10 @@ def run_gpu(args, cfg, rank, world, local_rank):
                         "graph_ms_per_step": graph_ms},
             "cpu_baseline": cpu,
             "bf16_cublas_graph": comparator,
+            "configs": configs,
             "setup_s": round(setup_s, 1),
         }
         print(json.dumps(line), flush=True)
-    model.close()
 
 
 # ------------------------------------------------------------------------------------------------
@@ -558,6 +646,7 @@ def main():
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-comparator", action="store_true", help="skip the torch bf16 CUDA-graph comparator")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other named shapes (measured after the headline)")
     ap.add_argument("--kv-block", type=int, default=0, help="amk_options.kv_block (minimum positions per attention chunk)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (smaller cases for profiler captures; not a bench line)")

@@ -726,7 +726,17 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
   if (op == OP_QKV)
     for (int i = tid; i < p.hd; i += kConsumerThreads) resid_rows[i] = __ldg(p.rope + (size_t)p.pos * p.hd + i);
 
+  // the RMSNorm gain vector (static) into the GEMV partial-sum region before the wait, so the
+  // thread's gains come from shared memory after it (no second round trip behind the inputs)
+  const int K = g.K;
+  const bool gain_smem = norm && K * 2 <= kPartBytes;
+  uint16_t* const gsm = reinterpret_cast<uint16_t*>(s.part);
+  if (gain_smem)
+    for (int i = tid * 8; i < K; i += 8 * kConsumerThreads)
+      *reinterpret_cast<uint4*>(gsm + i) = __ldg(reinterpret_cast<const uint4*>(gain + i));
+
   if (p.sync && first && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
+  else if (gain_smem) bar_compute();
   if (tr && tid == 0) tr[2] = globaltimer();
 
   // ---- inputs: this thread's own elements (tagged bf16 pairs, read through L1 right after the
@@ -841,9 +851,23 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
 #pragma unroll
       for (int c = 0; c < NP; ++c) {
         float* xp = &xv[(j * NP + c) * PE];
-        if (ok[j]) {   // the gains: read-only, a second (L1 / L2-hit) round trip after the inputs
+        if (ok[j]) {   // the gains: from shared memory when staged, else a second round trip
           uint32_t gp[PE / 2];
-          ld_bf16_words<PE>(gain + elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c)), gp);
+          const int e = elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c));
+          if (gain_smem) {
+            if constexpr (PE >= 8) {
+#pragma unroll
+              for (int k = 0; k < PE / 8; ++k) {
+                const uint4 w = reinterpret_cast<const uint4*>(gsm + e)[k];
+                gp[4 * k] = w.x; gp[4 * k + 1] = w.y; gp[4 * k + 2] = w.z; gp[4 * k + 3] = w.w;
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < PE / 2; ++k) gp[k] = reinterpret_cast<const uint32_t*>(gsm + e)[k];
+            }
+          } else {
+            ld_bf16_words<PE>(gain + e, gp);
+          }
 #pragma unroll
           for (int k = 0; k < PE; ++k) ss = fmaf(xp[k], xp[k], ss);
 #pragma unroll
@@ -902,6 +926,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
     if (tid < nrows) resid_rows[tid] = rv0;
     if (tid + kConsumerThreads < nrows) resid_rows[tid + kConsumerThreads] = rv1;
   }
+  if (gain_smem) bar_compute();   // every thread has its gains before the rows' partial sums reuse the region
   if (tr && tid == 0) {   // stamped once the (quantised) inputs exist
     if constexpr (IQ) asm volatile("" ::"f"(asc[0]));
     tr[4] = globaltimer();

@@ -39,7 +39,7 @@ constexpr int kThreads         = kConsumerThreads + 32;    // + 1 producer (bulk
 #define AMK_SLOTS 3
 #endif
 #ifndef AMK_INFLIGHT
-#define AMK_INFLIGHT 2
+#define AMK_INFLIGHT 1
 #endif
 constexpr int kSlotBytes       = AMK_SLOT_BYTES;           // one bulk-copy ring slot
 constexpr int kSlots           = AMK_SLOTS;                // ring depth
@@ -152,6 +152,7 @@ struct Task {
 };
 constexpr uint32_t kFirstOfStage = 1u;
 constexpr uint32_t kLastOfStage = 2u;
+constexpr uint32_t kTagWait = 4u;      // no counter: the task polls the tags of its (small) inputs
 
 // How one GEMV shape maps onto the 512 compute threads. A row of `rb` bytes is cut into groups of
 // `gb` bytes (one shared-memory vector load per thread); `wg_total` warps' worth of groups cover a

@@ -192,18 +192,19 @@ int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::s
   for (int b = 0; b < grid; ++b) {
     p.off[b] = (int)p.tasks.size();
     for (int l = 0; l < L; ++l) {
-      gemv_tasks(p.tasks, OP_QKV, l, s_qkv[b], l ? ctr_index(l - 1, CTR_DOWN) : -1, l ? grid : 0,
-                 ctr_index(l, CTR_QKV));
+      // QKV signals no counter: an attention task reads only its own KV head's q, k and v (a few
+      // KB) and polls their tags, so it starts when those rows are out, not when every CTA is done
+      gemv_tasks(p.tasks, OP_QKV, l, s_qkv[b], l ? ctr_index(l - 1, CTR_DOWN) : -1, l ? grid : 0, -1);
       for (int i = b; i < Hkv * cmax; i += grid) {
         Task t{};
         t.op = OP_ATTN;
         t.layer = (uint16_t)l;
         t.a = i % Hkv;
         t.b = i / Hkv;
-        t.wait_ctr = ctr_index(l, CTR_QKV);
-        t.wait_mult = grid;
+        t.wait_ctr = -1;
+        t.wait_mult = 0;
         t.sig_ctr = ctr_index(l, CTR_ATTN);   // signalled by the merging (last-arriving) chunk
-        t.flags = (i == b ? kFirstOfStage : 0) | (i + grid >= Hkv * cmax ? kLastOfStage : 0);
+        t.flags = kTagWait | (i == b ? kFirstOfStage : 0) | (i + grid >= Hkv * cmax ? kLastOfStage : 0);
         p.tasks.push_back(t);
       }
       gemv_tasks(p.tasks, OP_O, l, s_o[b], ctr_index(l, CTR_ATTN), Hkv, ctr_index(l, CTR_O));
@@ -318,13 +319,19 @@ int check_plan(const amk_dims& d, const Plan& p, std::string* msg) {
       if ((int)t.wait_mult != producers[t.wait_ctr])
         return fail(fmt("counter %ld: threshold %ld does not join all %ld producers", t.wait_ctr, t.wait_mult, producers[t.wait_ctr]));
     }
-  // every stage after the first waits on its predecessor (happens-before of every input)
+  // every stage after the first waits on its predecessor: on its counter, or (attention, whose
+  // inputs are one KV head's q, k and v) on the tags of the same layer's QKV output
   for (int b = 0; b < grid; ++b)
     for (int i = p.off[b]; i < p.off[b + 1]; ++i) {
       const Task& t = p.tasks[i];
+      if (t.op == OP_ATTN) {
+        if (!(t.flags & kTagWait) || t.wait_ctr != -1)
+          return fail(fmt("CTA %ld task %ld: an attention task must poll its inputs' tags", b, i - p.off[b]));
+        continue;
+      }
+      if (t.flags & kTagWait) return fail(fmt("CTA %ld task %ld: only attention polls tags", b, i - p.off[b]));
       if (!(t.flags & kFirstOfStage) || (t.op == OP_QKV && t.layer == 0)) continue;
       int want = t.op == OP_QKV ? ctr_index(t.layer - 1, CTR_DOWN)
-               : t.op == OP_ATTN ? ctr_index(t.layer, CTR_QKV)
                : t.op == OP_O ? ctr_index(t.layer, CTR_ATTN)
                : t.op == OP_GU ? ctr_index(t.layer, CTR_O)
                : t.op == OP_DOWN ? ctr_index(t.layer, CTR_GU)

@@ -10,7 +10,7 @@ from decode_megakernel_launch_b200 import sweep as S
 
 def test_compile_defaults_match_the_header():
     d = S.compile_defaults()
-    assert d["AMK_SLOT_BYTES"] == 65536 and d["AMK_SLOTS"] == 3 and d["AMK_INFLIGHT"] == 2
+    assert d["AMK_SLOT_BYTES"] == 65536 and d["AMK_SLOTS"] == 3 and d["AMK_INFLIGHT"] == 1
     assert set(d) == set(B.TUNABLE)
     for k, v in d.items():
         assert v in B.TUNABLE[k], (k, v)
