@@ -20,7 +20,7 @@ def _newest_source_mtime() -> float:
 # Compile-time knobs of the kernel (macros of csrc/amk_internal.h) that a variant build may set,
 # with the values the kernel's static checks and the planner accept.
 TUNABLE = {
-    "AMK_SLOT_BYTES": (32768, 49152, 65536),   # ring slot size (the ring and the 64 KB input stage share 227 KB)
+    "AMK_SLOT_BYTES": (32768, 49152, 65536),   # ring slot size (3 slots of 64 KB fill shared memory)
     "AMK_SLOTS": (2, 3, 4, 5, 6),             # ring depth (static_assert bounds the total)
     "AMK_INFLIGHT": (1, 2, 3, 4),             # outstanding bulk copies (<= slots)
     "AMK_PF_ITEMS": tuple(range(0, 17)),      # L2 warm-up items while the compute warps stall

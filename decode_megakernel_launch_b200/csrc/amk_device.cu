@@ -688,7 +688,7 @@ __device__ __forceinline__ int piece_offset(int col, int lane, int c) {
 template <int WK>
 __device__ __forceinline__ int elem_of_byte(int b) { return WK == 0 ? b / 2 : WK == 1 ? b : b * 2; }
 
-template <int WK, int GB, int NR>
+template <int WK, int GB, int NR, bool PART = (WK == 2)>
 __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uint32_t it, int token,
                                              unsigned long long* tr) {
   const Smem s = smem_view();
@@ -713,12 +713,19 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
   const uint16_t* sc = IQ ? gemv_scales(p, op, l) : nullptr;
   if (IQ && sc)
     for (int i = tid; i < nrows; i += kConsumerThreads) s.scale[i] = bf2f(__ldg(sc + row0 + i));
-  bool ok[NR];
+  // pv: this thread's pieces that lie in the row. PART: the last warp of a row may be partly
+  // filled, so each piece is checked against the row's end; otherwise whole groups are. Only int4
+  // rows can end inside a warp: rows are multiples of 64 elements, so an int8 or bf16 row is a
+  // whole number of warps of the smallest group, and the planner picks no larger group that leaves
+  // lanes idle when a smaller one fills them.
+  bool pv[NR * NP];
   int col[NR];
 #pragma unroll
   for (int j = 0; j < NR; ++j) {
     col[j] = j * g.wpg + wg;
-    ok[j] = active && j < g.nr && col[j] < g.wg_total;
+    const bool ok = active && j < g.nr && col[j] < g.wg_total;
+#pragma unroll
+    for (int c = 0; c < NP; ++c) pv[j * NP + c] = PART ? ok && piece_offset<GB>(col[j], lane, c) < g.rb : ok;
   }
   const uint16_t* gain =
       op == OP_QKV ? p.layers[l].attn_norm : op == OP_GU ? p.layers[l].ffn_norm : op == OP_LM ? p.final_norm : nullptr;
@@ -780,7 +787,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
       for (int c = 0; c < NP; ++c) {
         float* xp = &xv[(j * NP + c) * PE];
         const int e = elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c));
-        if (ok[j]) {
+        if (pv[j * NP + c]) {
           uint32_t ew[PE / 2];
           ld_bf16_words<PE>(erow + e, ew);
 #pragma unroll
@@ -795,9 +802,8 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
     constexpr int LPP = PE >= 4 ? PE / 4 : 1;
 #pragma unroll
     for (int k = 0; k < NL; ++k) {
-      const int j = (k / LPP) / NP;
       wv[k] = make_uint4(0u, tag_in, 0u, tag_in);
-      if (ok[j]) {
+      if (pv[k / LPP]) {
         if constexpr (PE >= 4) {
           wv[k] = ld_words2_ca(waddr(k));
         } else {
@@ -851,7 +857,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
 #pragma unroll
       for (int c = 0; c < NP; ++c) {
         float* xp = &xv[(j * NP + c) * PE];
-        if (ok[j]) {   // the gains: from shared memory when staged, else a second round trip
+        if (pv[j * NP + c]) {   // the gains: from shared memory when staged, else a second round trip
           uint32_t gp[PE / 2];
           const int e = elem_of_byte<WK>(piece_offset<GB>(col[j], lane, c));
           if (gain_smem) {
@@ -955,9 +961,10 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
             const uint8_t* rowp = sbuf + (size_t)(r + rr) * g.rb;
 #pragma unroll
             for (int j = 0; j < NR; ++j) {
-              if (ok[j]) {
+              if (pv[j * NP]) {   // a group's pieces are contiguous: the first lies in the row if any does
 #pragma unroll
-                for (int c = 0; c < NP; ++c) {
+              for (int c = 0; c < NP; ++c) {
+                if (!PART || c == 0 || pv[j * NP + c]) {
                   uint32_t w[WPP];
                   lds_group<PB>(rowp + piece_offset<GB>(col[j], lane, c), w);
                   if constexpr (WK == 1) {
@@ -999,6 +1006,7 @@ __device__ __forceinline__ uint32_t gemv_body(const Params& p, const Task t, uin
                     v += f2sum(acc2);
                   }
                 }
+              }
               }
             }
           }
@@ -1567,7 +1575,7 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
 #endif
           case 16:
 #if AMK_INLINE_HOT4
-            if (g.nr <= 1) { it = gemv_body<2, 16, 1>(p, t, it, token, tr); break; }
+            if (g.nr <= 1 && g.rb % (32 * 16) == 0) { it = gemv_body<2, 16, 1, false>(p, t, it, token, tr); break; }
 #endif
             it = gemv_nr<2, 16>(p, t, it, token, tr, g.nr); break;
           case 8: it = gemv_nr<2, 8>(p, t, it, token, tr, g.nr); break;

@@ -154,15 +154,15 @@ constexpr uint32_t kFirstOfStage = 1u;
 constexpr uint32_t kLastOfStage = 2u;
 constexpr uint32_t kTagWait = 4u;      // no counter: the task polls the tags of its (small) inputs
 
-// How one GEMV shape maps onto the 512 compute threads. A row of `rb` bytes is cut into groups of
+// How one GEMV shape maps onto the compute threads. A row of `rb` bytes is cut into groups of
 // `gb` bytes (one shared-memory vector load per thread); `wg_total` warps' worth of groups cover a
-// row. Warps form `rp` row groups of `wpg` warps; a thread keeps the activations of its groups in
+// row (the lanes of the last warp past the row's end stay idle). Warps form `rp` row groups of `wpg` warps; a thread keeps the activations of its groups in
 // registers for the whole task (`nr` groups per thread).
 struct GemvGeom {
   int32_t K;         // elements per row
   int32_t rb;        // bytes per row
-  int32_t gb;        // bytes per group: 16, 8, 4 or 2
-  int32_t wg_total;  // (rb / gb) / 32
+  int32_t gb;        // bytes per group: 64, 32, 16, 8, 4 or 2
+  int32_t wg_total;  // ceil((rb / gb) / 32): warps of groups per row (the last one may be partly filled)
   int32_t wpg;       // warps per row group
   int32_t nr;        // groups per thread
   int32_t rp;        // row groups

@@ -122,6 +122,11 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
   // ---- (re)load the plan, layer pointers and RoPE table when the model differs ----
   std::vector<const void*> ptrs = pointer_list(d, *w);
   if (!S.loaded || !same_dims(S.dims, d) || S.ptrs != ptrs) {
+    // a reload copies from pageable host memory, which stream capture does not allow: refuse it
+    // before enqueuing anything (a capture would be invalidated)
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return AMK_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return AMK_ERR_INVALID_ARG;
     S.loaded = false;
     const int grid = S.sms;
     Plan pl;

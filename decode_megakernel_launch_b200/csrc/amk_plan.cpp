@@ -73,14 +73,19 @@ bool make_geom(int K, int wk, GemvGeom* g) {
   for (int i = 0; i < 6; ++i) {
     const int gb = gbs[i];
     if (gb > max_bytes || gb < min_bytes) continue;
-    if (rb % (gb * 32) != 0) continue;
-    int W = rb / gb / 32;
+    if (rb % gb != 0) continue;
+    // groups of a row over whole warps; an int4 row's last warp may be partly filled (its idle
+    // lanes count against the candidate); int8 and bf16 rows always have a whole-warp choice
+    const int groups = rb / gb;
+    if (wk != AMK_W_INT4 && groups % 32) continue;
+    int W = (groups + 31) / 32;
+    const double lane_util = double(groups) / (W * 32);
     int nr = (W + kConsumerWarps - 1) / kConsumerWarps;
     if (nr > max_bytes / gb) continue;
     int wpg = W < kConsumerWarps ? W : kConsumerWarps;
     int rp = nr == 1 ? kConsumerWarps / wpg : 1;
     double bal = nr == 1 ? double(rp * wpg) / kConsumerWarps : double(W) / (nr * kConsumerWarps);
-    double score = bal * eff[i];
+    double score = bal * eff[i] * lane_util;
     if (score > best + 1e-9) {
       best = score;
       // rows per slot: a power of two below 8, else a multiple of 8, so every 128-row epilogue block

@@ -85,11 +85,9 @@ PRESETS = {
     "llama1b_long32k": ModelConfig("llama1b_long32k", 4, 16, 2048, 32, 8, 64, 8192, 128256, True, 5e5,
                                    prefill_len=32768, decode_steps=64, compare_steps=4),
 }
-# W4A16 variants of the same shapes (int4 weight-only, per-row bf16 scales). The int4 GEMV wants
-# rows of a multiple of 256 elements, so the tiny variant's FFN is 768 wide instead of 704.
+# W4A16 variants of the same shapes (int4 weight-only, per-row bf16 scales).
 for _n in ("tiny", "llama1b", "llama8b"):
     PRESETS[_n + "_int4"] = PRESETS[_n].with_(name=_n + "_int4", weight_dtype="int4")
-PRESETS["tiny_int4"] = PRESETS["tiny_int4"].with_(ffn=768)
 
 
 def preset(name: str, **overrides) -> ModelConfig:

@@ -195,11 +195,14 @@ const char* amk_last_cuda_error(void);
  * with 1152 positions needs ~1.8 MiB). The first call on a device (with that device current) looks up
  * the array's device address (cudaGetSymbolAddress) and sets the kernel's attributes; make that first
  * call before any stream capture. Every call shares the array, which keeps the last call's contents:
- * each call zeroes the counters and status words on `stream` and re-uploads the task list, layer
- * pointers and RoPE table when dims or pointers differ from the previous call on that device. Calls
- * whose launches overlap on the GPU (unordered streams) race on the array and must be serialized by
- * the caller. A wait that expires inside such a launch is not reported (use amk_decode_step and
- * amk_status for the sticky status). */
+ * each call zeroes the counters and status words on `stream` and reloads the task list, layer
+ * pointers and RoPE table (from pageable host memory) when dims or pointers differ from the previous
+ * call on that device; such a reload is refused with AMK_ERR_INVALID_ARG while `stream` is capturing,
+ * so every call that changes dims or pointers must also come before any capture. Calls whose
+ * launches overlap on the GPU (unordered streams) race on the array and must be serialized by the
+ * caller. A wait that expires inside such a launch is not reported, and neither is a next token read
+ * back (token_id = -1) that lies outside [0, V): the kernel then decodes token 0 (use
+ * amk_decode_step and amk_status for the sticky status). */
 int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* weights, int token_id, int pos,
                             float* logits_out, int* next_token_out, void* stream);
 

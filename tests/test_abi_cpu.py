@@ -98,12 +98,16 @@ def test_unsupported_dims_rejected():
     assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
 
 
-def test_int4_rows_must_be_a_multiple_of_256():
-    # the int4 GEMV reads at least one 32-bit word of nibbles per lane: rows of 256 elements
+def test_int4_rows_need_only_the_common_multiple_of_64():
+    # int4 rows that no whole number of warps covers run with the last warp partly idle
     d = dims_of(synth.preset("tiny_int4"))
     assert amk.plan_check(d, 148)[0] == amk.AMK_OK
-    d.ffn = 704
+    for k in (704, 320, 64):
+        d.ffn = k
+        assert amk.plan_check(d, 148)[0] == amk.AMK_OK, k
+    d.ffn = 672 + 2                                   # not a multiple of 64
     assert amk.plan_check(d, 148)[0] == amk.AMK_ERR_UNSUPPORTED
+    d.ffn = 704
     d.weight_dtype = amk.AMK_W_INT8
     assert amk.plan_check(d, 148)[0] == amk.AMK_OK
     d = dims_of(synth.preset("tiny"))

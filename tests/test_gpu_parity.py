@@ -193,6 +193,9 @@ ODD = [
     # int4 weights with a tied (bf16) head, head_dim 128, one KV head
     synth.ModelConfig("odd_int4_tied", 25, 2, 256, 2, 1, 128, 1280, 515, True, 5e5, prompt_len=5,
                       decode_steps=20, compare_steps=20, weight_dtype="int4"),
+    # int4 rows that no whole number of warps covers: d 320 (160 bytes), ffn 448 (224 bytes)
+    synth.ModelConfig("odd_int4_k320", 26, 2, 320, 5, 5, 64, 448, 999, False, 1e4, prompt_len=6,
+                      decode_steps=10, compare_steps=10, weight_dtype="int4"),
 ]
 
 
