@@ -26,6 +26,7 @@ TUNABLE = {
     "AMK_PF_ITEMS": tuple(range(0, 17)),      # L2 warm-up items while the compute warps stall
     "AMK_PF_GAP_NS": (200, 400, 600, 800, 1000, 1200, 1600),
     "AMK_PF_STALL_NS": (100, 200, 400, 800),
+    "AMK_PF_CONTINUOUS": (0, 1),              # warm-up between stalls too
     "AMK_NB32": (2, 4),                       # rows per register batch, 32-byte groups
     "AMK_I4_NOSHIFT": (0, 1),                 # int4 high nibbles in place (1) or shifted (0)
     "AMK_CONSUMER_WARPS": (12, 15, 16),       # compute warps per CTA (16 caps registers at 96)

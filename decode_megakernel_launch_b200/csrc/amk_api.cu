@@ -22,8 +22,49 @@ cudaError_t launch_pack(int role, int hd, int ffn, const void* src, int src_dtyp
 using namespace amk;
 
 namespace {
-
 thread_local std::string g_cuda_error;
+}
+
+namespace amk {
+
+int encode_kv_maps(Params& p) {
+  using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeTiled encode = nullptr;
+  if (!encode) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f) {
+      g_cuda_error = "cuTensorMapEncodeTiled: not available from the driver";
+      return AMK_ERR_CUDA;
+    }
+    encode = reinterpret_cast<EncodeTiled>(f);
+  }
+  // [L * Hkv * max_seq rows][hd] bf16; boxes of 64 elements (128 bytes) by 64 or 16 rows, swizzled
+  // so that the rows of an 8-row tile fall in distinct bank groups; rows past the end read as zero
+  const cuuint64_t dims[2] = {(cuuint64_t)p.hd, (cuuint64_t)p.L * p.Hkv * p.max_seq};
+  const cuuint64_t strides[1] = {(cuuint64_t)p.hd * 2};
+  const cuuint32_t unit[2] = {1, 1};
+  for (int b = 0; b < 2; ++b) {
+    const cuuint32_t box[2] = {64, b ? 16u : 64u};
+    for (int i = 0; i < 2; ++i) {
+      const CUresult r = encode(i ? &p.vmap[b] : &p.kmap[b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, i ? p.vcache : p.kcache,
+                                dims, strides, box, unit, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) {
+        g_cuda_error = "cuTensorMapEncodeTiled refused the KV cache layout (error " + std::to_string((int)r) + ")";
+        return AMK_ERR_CUDA;
+      }
+    }
+  }
+  return AMK_OK;
+}
+
+}  // namespace amk
+
+namespace {
 
 int cuda_fail(cudaError_t e, const char* what) {
   g_cuda_error = std::string(what) + ": " + cudaGetErrorString(e);
@@ -247,6 +288,7 @@ int amk_create(const amk_dims* dims, const amk_weights* w, const amk_options* op
   p.lm_s = (!d.tied_head && i8) ? static_cast<const uint16_t*>(w->slm) : nullptr;
   p.kcache = static_cast<uint16_t*>(w->k_cache);
   p.vcache = static_cast<uint16_t*>(w->v_cache);
+  if ((rc = encode_kv_maps(p))) return fail(rc);
   for (int i = 0; i < 5; ++i) p.geom[i] = pl.geom[i];
   p.kv_block = h->opt.kv_block > 0 ? h->opt.kv_block : 64;
   p.kv_chunks_max = pl.kv_chunks_max;

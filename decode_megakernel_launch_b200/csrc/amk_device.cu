@@ -73,6 +73,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
 }
+// One tile of a 2-D tensor map (x: column, a multiple of 16 bytes; y: row) into shared memory.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -203,7 +210,7 @@ struct Smem {
   Misc* misc;
 };
 
-extern __shared__ __align__(128) uint8_t smem_raw[];
+extern __shared__ __align__(1024) uint8_t smem_raw[];   // 1024: the 128-byte swizzle's period
 __device__ __forceinline__ Smem smem_view();
 
 __device__ __forceinline__ Smem carve(uint8_t* base) {
@@ -383,7 +390,7 @@ __device__ __forceinline__ void task_range(const Params& p, const Task& t, int& 
 // are the item's byte ranges (n1 = 0 for GEMV items; n0 = n1 = 0 for an attention block that holds
 // only the current position, which is written this step and patched in shared memory).
 __device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor& c, const uint8_t*& src0,
-                          uint32_t& n0, const uint8_t*& src1, uint32_t& n1) {
+                          uint32_t& n0, const uint8_t*& src1, uint32_t& n1, int& trow, int& tn) {
   while (c.ti < nt) {
     const Task& t = tasks[c.ti];
     if (!c.started) {
@@ -401,10 +408,15 @@ __device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor
         const int nps = attn_positions_per_slot(p.hd);
         const int blk = c.sub, be = min(blk + nps, c.end);
         const int ntma = max(0, min(be, p.pos) - blk);
-        const size_t off = (((size_t)t.layer * p.Hkv + t.a) * p.max_seq + blk) * p.hd;
+        const size_t row = ((size_t)t.layer * p.Hkv + t.a) * p.max_seq + blk;
+        const size_t off = row * p.hd;
+        // the contiguous rows already in the cache (for the L2 warm-up); the copy itself moves
+        // 16-row tensor boxes of rows blk..be-1 (the current position's row is patched in later)
         src0 = reinterpret_cast<const uint8_t*>(p.kcache + off);
         src1 = reinterpret_cast<const uint8_t*>(p.vcache + off);
         n0 = n1 = (uint32_t)ntma * (uint32_t)p.hd * 2u;
+        trow = (int)row;
+        tn = be - blk;
         c.sub = be;
       } else {
         const int n = min(c.rs, c.end - c.sub);
@@ -412,6 +424,7 @@ __device__ bool next_item(const Params& p, const Task* tasks, int nt, ItemCursor
         n0 = (uint32_t)n * (uint32_t)c.rb;
         src1 = nullptr;
         n1 = 0;
+        tn = 0;
         c.sub += n;
       }
       return true;
@@ -428,6 +441,7 @@ __device__ __forceinline__ void prefetch_line_l2(const void* a) {
 __device__ __forceinline__ void prefetch_bulk_l2(const void* a, uint32_t bytes) {   // 16-B aligned, 16-B multiple
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(bytes) : "memory");
 }
+
 
 // L2 prefetch of the small static data a task reads on its critical path (row scales, RMSNorm gain,
 // this position's RoPE row, the embedding row), issued when the producer starts streaming the
@@ -453,9 +467,14 @@ __device__ void prefetch_side_data(const Params& p, const Task& t, int token) {
 }
 
 // Producer lane: issues every item of the CTA's byte stream into the ring in order, gated only by
+
 // the ring's empty barriers (never by other CTAs).
 __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt) {
   Smem s = smem_view();
+  if (smem_u32(s.ring) & 1023u) {   // the swizzled tensor copies need the 1024-byte period
+    raise_abort(p, 7u << 16);
+    return;
+  }
   const uint64_t pol = policy_evict_first();
   int token = p.token;
   if (token < 0) token = __ldcg(p.next_token);
@@ -465,8 +484,10 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
   int last_task = -1;
   const uint8_t *a0, *a1;
   uint32_t n0, n1;
+  int trow, tn;
+  uint64_t last_pf = 0;
   bool first_item = false;
-  while (next_item(p, tasks, nt, cur, a0, n0, a1, n1)) {
+  while (next_item(p, tasks, nt, cur, a0, n0, a1, n1, trow, tn)) {
     if (cur.ti != last_task) {
       last_task = cur.ti;
       first_item = true;
@@ -483,7 +504,7 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
         // the slot's previous item has landed but is still held: once that lasts kStallNs the
         // compute warps are waiting on a counter, so warm L2 with what follows, paced
         const uint64_t t0 = globaltimer();
-        uint64_t last = 0;
+        uint64_t& last = last_pf;
         bool cur_warm = pf_it > it + 1;   // already warmed as a look-ahead item of an earlier stall
         // non-blocking probes: a suspended try_wait would hold the producer past the warm-up times
         while (!mbar_test_wait(&s.empty[slot], par)) {
@@ -497,12 +518,13 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
               mbar_test_wait(&s.full[slot], par)) {
             const uint8_t *b0, *b1;
             uint32_t m0, m1;
+            int r0, rn;
             if (!cur_warm) {   // this item first: it is copied as soon as the slot frees
               if (n0) prefetch_bulk_l2(a0, n0);
               if (n1) prefetch_bulk_l2(a1, n1);
               cur_warm = true;
               last = now;
-            } else if (next_item(p, tasks, nt, pfc, b0, m0, b1, m1)) {
+            } else if (next_item(p, tasks, nt, pfc, b0, m0, b1, m1, r0, rn)) {
               if (m0) prefetch_bulk_l2(b0, m0);
               if (m1) prefetch_bulk_l2(b1, m1);
               ++pf_it;
@@ -526,7 +548,23 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
       p.trace[((size_t)blockIdx.x * p.max_tasks_per_cta + cur.ti) * AMK_TRACE_WORDS + 8] = globaltimer();
       first_item = false;
     }
-    if (n0 + n1 > 0) {
+    if (tn > 0) {
+      // attention keys and values: each 64-column half as 64-row boxes, the last rows as 16-row
+      // boxes (rows past the item are loaded too and masked by the consumer), 128-byte swizzled
+      const int nbig = tn >> 6, nsmall = ((tn & 63) + 15) >> 4, nh = p.hd >> 6;
+      const int nps = attn_positions_per_slot(p.hd);
+      uint8_t* const kb = s.ring + slot * kSlotBytes;
+      mbar_expect_tx(&s.full[slot], (uint32_t)nh * 2u * (uint32_t)(nbig * 8192 + nsmall * 2048));
+      for (int hh = 0; hh < nh; ++hh) {
+        for (int b = 0; b < nbig + nsmall; ++b) {
+          const bool big = b < nbig;
+          const int r = big ? 64 * b : 64 * nbig + 16 * (b - nbig);
+          const uint32_t o = (uint32_t)(hh * nps * 128 + r * 128);
+          tma_load_2d(kb + o, &p.kmap[big ? 0 : 1], hh * 64, trow + r, &s.full[slot], pol);
+          tma_load_2d(kb + kSlotBytes / 2 + o, &p.vmap[big ? 0 : 1], hh * 64, trow + r, &s.full[slot], pol);
+        }
+      }
+    } else if (n0 + n1 > 0) {
       mbar_expect_tx(&s.full[slot], n0 + n1);
       bulk_g2s(s.ring + slot * kSlotBytes, a0, n0, &s.full[slot], pol);
       if (n1) bulk_g2s(s.ring + slot * kSlotBytes + kSlotBytes / 2, a1, n1, &s.full[slot], pol);
@@ -536,6 +574,25 @@ __device__ __noinline__ void producer(const Params& p, const Task* tasks, int nt
     if (p.trace && cur.sub >= cur.end)   // the task's last item is issued
       p.trace[((size_t)blockIdx.x * p.max_tasks_per_cta + cur.ti) * AMK_TRACE_WORDS + 9] = globaltimer();
     ++it;
+    // the warm-up also runs between stalls, one item per kPfGapNs and at most kPfItems ahead of
+    // the ring, so HBM already streams what the ring copies next (they then mostly hit L2)
+    if (kPfContinuous && kPfItems > 0 && pf_it < it + kPfItems && pf_it != 0xffffffffu) {
+      const uint64_t now = globaltimer();
+      if (now - last_pf > kPfGapNs) {
+        const uint8_t *b0, *b1;
+        uint32_t m0, m1;
+        int r0, rn;
+        if (pf_it <= it) { pfc = cur; pf_it = it; }
+        if (next_item(p, tasks, nt, pfc, b0, m0, b1, m1, r0, rn)) {
+          if (m0) prefetch_bulk_l2(b0, m0);
+          if (m1) prefetch_bulk_l2(b1, m1);
+          ++pf_it;
+          last_pf = now;
+        } else {
+          pf_it = 0xffffffffu;
+        }
+      }
+    }
   }
 }
 
@@ -1166,6 +1223,45 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 __device__ __forceinline__ float exp2_scale(float m, float M) { return m == -CUDART_INF_F ? 0.f : fast_exp2(m - M); }
 
+// ---- warp-level tensor-core helpers (attention) ----
+// D += A B for one m16n8k16 tile: bf16 A (4 registers: rows g / g + 8, k 2t.. / 2t + 8..) and B
+// (2 registers: k 2t.. / 2t + 8.., column g), fp32 D (rows g / g + 8, columns 2t, 2t + 1), where g =
+// lane / 4 and t = lane % 4.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Four 8x8 bf16 tiles from shared memory; lanes 8i..8i+7 give the row addresses of tile i.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+// Two 8x8 bf16 tiles, transposed; lanes 0..15 give the row addresses.
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
+// (a, b) as a bf16 pair (a in the low half) plus the bf16 pair of what rounding left over, so that
+// hi + lo carries about 16 significant bits of each value.
+__device__ __forceinline__ void split_bf2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+  const __nv_bfloat162 l2 = __floats2bfloat162_rn(a - __low2float(h2), b - __high2float(h2));
+  hi = *reinterpret_cast<const uint32_t*>(&h2);
+  lo = *reinterpret_cast<const uint32_t*>(&l2);
+}
+// Float <-> int keys whose signed order is the float order (for an integer atomicMax).
+__device__ __forceinline__ int max_key(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float key_max(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7fffffff); }
+// Byte offset of 16-byte chunk ch (8 elements) of row r of a key or value plane in a ring slot. The
+// tensor copies land 64-column halves (128-byte rows, nps rows each) one after the other, with the
+// 128-byte swizzle: chunk c of row r sits at chunk c ^ (r % 8).
+__device__ __forceinline__ uint32_t kv_off(int r, int ch, int nps) {
+  return (uint32_t)((ch >> 3) * nps * 128 + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
 // Log-sum-exp merge of the C chunk partials (unnormalised o, running max m in log2 units, sum l) of
 // KV head h of layer l into the tagged attention output. One thread per (query head, element); a
 // warp holds 32 elements of one query head. Per block of 16 chunks, lane k < 16 loads chunk k's
@@ -1218,16 +1314,21 @@ __device__ __noinline__ void merge_head(const Params& p, int h, int C, int l) {
   }
 }
 
-// Split-KV flash decoding of one (KV head, chunk) task. The compute warps form NHG groups, one per
-// pair of query heads of this KV head's GQA group (kHeadsPerWarp = 2 keeps a warp's running state
-// small: 2 x (max, sum, 8 outputs) per lane). Inside a warp, LPP lanes hold one 16-byte piece of a
-// key/value row (8 elements) and PPW positions are processed per step; each sub-warp keeps an online
-// softmax, merged across sub-warps by shuffles and across the group's warps by a shared-memory tree.
-#ifndef AMK_HEADS_PER_WARP
-#define AMK_HEADS_PER_WARP 2
-#endif
-constexpr int kHeadsPerWarp = AMK_HEADS_PER_WARP;
-
+// Split-KV flash decoding of one (KV head, chunk) task on the tensor cores. The chunk's keys and
+// values arrive in the ring as 128-byte-swizzled tiles (kv_off), so every ldmatrix below is free of
+// bank conflicts. Per ring slot:
+//   QK:  S = q K^T with mma.m16n8k16 (bf16 in, fp32 accumulate). The A operand holds the query heads
+//        of this KV head's group in rows 0..G-1 and the bf16 residual of the same heads in rows
+//        8..8+G-1, so q enters as hi + lo (~16 significant bits) while the keys stay exact bf16;
+//        warps take 8-position tiles, write S to shared memory and their per-head maxima.
+//   softmax: the slot maximum joins the running maximum M (log2 units: q is pre-scaled by
+//        log2(e)/sqrt(hd)); P = 2^(S - M), split the same way into hi/lo rows of the P tile.
+//   PV:  O += P V with mma.m16n8k16, warps over 8-dimension output tiles (and over position steps
+//        when there are more warps than tiles); the running sum l comes from one more MMA against a
+//        tile of ones, so l and O see the same P. O and l are rescaled by 2^(M_old - M) first.
+// The chunk's (O, M, l) is written as its partial; the last chunk of the head to arrive merges them.
+// The contraction is tiny (at most 4 query rows per KV head), so the legacy warp-level MMA serves:
+// it replaces the per-lane FMA and shuffle work, which was the cost here, and needs no TMEM.
 #ifndef AMK_INLINE_ATTN
 #define AMK_INLINE_ATTN 0
 #endif
@@ -1239,17 +1340,12 @@ __device__ __noinline__
 #endif
 uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long long* tr) {
   const Smem s = smem_view();
-  constexpr int LPP = HD * 2 / 16;       // lanes per position (one 16-byte piece each)
-  constexpr int PPW = 32 / LPP;          // positions per warp step
-  constexpr int NPS = kSlotBytes / (4 * HD);
-  constexpr int HW = kHeadsPerWarp;
+  constexpr int NPS = kSlotBytes / (4 * HD);           // positions per ring slot (keys, then values)
+  static_assert(NPS % 16 == 0, "a slot holds whole 16-row tensor boxes");
+  static_assert(kMaxGroup * NPS * 4 + 2 * kMaxGroup * 4 + 16 * (NPS + 8) * 2 <= kAuxBytes,
+                "scores, slot maxima and the P tile fit aux");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cl = lane % LPP, sw = lane / LPP;
   const int G = p.Hq / p.Hkv;
-  const int NHG = (G + HW - 1) / HW;                 // head groups
-  const int WPH = kConsumerWarps / NHG;              // warps per head group (8 or 16)
-  const int hg = warp / WPH, wi = warp % WPH;
-  const bool in_group = hg < NHG;
   const int h = t.a, c = t.b, l = t.layer;
   const int P = p.pos + 1;
   const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
@@ -1289,106 +1385,166 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
     }
     if (ik < 2 * HD) kvc[(ik < HD ? 0 : HD) + unpack(ik % HD)] = f2bf(__uint_as_float(v[2].x));
   }
+  float* const Ssm = s.aux;                                      // [kMaxGroup][NPS] scores
+  int* const smax = reinterpret_cast<int*>(s.aux + kMaxGroup * NPS);   // [2][kMaxGroup] slot maxima (ordered keys)
+  uint8_t* const ptile = reinterpret_cast<uint8_t*>(smax + 2 * kMaxGroup);
+  constexpr int PSTR = (NPS + 8) * 2;                            // P tile row bytes (padded)
+  // the P tile's rows past the group's heads stay zero for the whole task
+  for (int i = tid; i < 16 * PSTR / 16; i += kConsumerThreads)
+    reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (tid < 2 * kMaxGroup) smax[tid] = max_key(-CUDART_INF_F);
   bar_compute();
+  if (tr && tid == 0) tr[10] = globaltimer();
 
-  float m[HW], ls[HW], o[HW][8];
-  float qr[HW][8];   // this lane's 8 query elements of each of its heads, for the whole task
-  const int g0 = hg * HW;                               // first query head of this warp's group
+  // q as the A operand (see above): fragments for the whole task
+  constexpr int KS = HD / 16;                          // k-steps of the QK contraction
+  const int gid = lane >> 2, t4 = lane & 3;
+  uint32_t qa[KS][4];
 #pragma unroll
-  for (int g = 0; g < HW; ++g) {
-    m[g] = -CUDART_INF_F;
-    ls[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
-    if (in_group && g0 + g < G) {
-      const float4 q0 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8);
-      const float4 q1 = *reinterpret_cast<const float4*>(qsm + (g0 + g) * HD + cl * 8 + 4);
-      qr[g][0] = q0.x; qr[g][1] = q0.y; qr[g][2] = q0.z; qr[g][3] = q0.w;
-      qr[g][4] = q1.x; qr[g][5] = q1.y; qr[g][6] = q1.z; qr[g][7] = q1.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qr[g][e] = 0.f;
+  for (int ks = 0; ks < KS; ++ks) {
+    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+    if (gid < G) {
+      const float* qq = qsm + gid * HD + 16 * ks + 2 * t4;
+      x0 = qq[0]; x1 = qq[1]; x2 = qq[8]; x3 = qq[9];
     }
+    split_bf2(x0, x1, qa[ks][0], qa[ks][1]);
+    split_bf2(x2, x3, qa[ks][2], qa[ks][3]);
   }
 
-  for (int blk = cb; blk < ce; blk += NPS, ++it) {
+  // PV jobs: (output tile of 8 dimensions, position-step residue); most configurations give one
+  // job per warp
+  constexpr int NTO = HD / 8;
+  constexpr int KSPLIT = kConsumerWarps / NTO > 1 ? kConsumerWarps / NTO : 1;
+  constexpr int NJOBS = NTO * KSPLIT;
+  constexpr int NJ = (NJOBS + kConsumerWarps - 1) / kConsumerWarps;
+  float acc[NJ][4], lacc[NJ][4];
+#pragma unroll
+  for (int jb = 0; jb < NJ; ++jb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[jb][i] = lacc[jb][i] = 0.f;
+  float Mrun[kMaxGroup];
+#pragma unroll
+  for (int g = 0; g < kMaxGroup; ++g) Mrun[g] = -CUDART_INF_F;
+
+  const uint32_t ptile_a = smem_u32(ptile);
+  constexpr uint32_t kOnes = 0x3f803f80u;                        // bf16 pair (1, 1)
+
+  for (int blk = cb, si = 0; blk < ce; blk += NPS, ++it, ++si) {
     const int slot = it % kSlots;
     wait_slot(p, &s.full[slot], (it / kSlots) & 1, (2u << 16) | slot);
+    if (tr && tid == 0 && blk == cb) tr[11] = globaltimer();
     const int n = min(blk + NPS, ce) - blk;
-    uint8_t* kb = s.ring + slot * kSlotBytes;
-    uint8_t* vb = kb + kSlotBytes / 2;
-    if (p.pos >= blk && p.pos < blk + n) {
-      // this step's own key/value row (not copied: the QKV stage writes it in this launch) from the
-      // staged copy; the proxy fence orders these generic writes before the slot's next bulk copy
-      const int j = p.pos - blk;
-      if (tid < HD / 4) {
-        reinterpret_cast<uint2*>(kb + (size_t)j * HD * 2)[tid] = reinterpret_cast<const uint2*>(kvc)[tid];
-        reinterpret_cast<uint2*>(vb + (size_t)j * HD * 2)[tid] = reinterpret_cast<const uint2*>(kvc + HD)[tid];
-        fence_proxy_async_smem();
+    const int KT = (n + 15) >> 4;                       // 16-position steps
+    uint8_t* const kb = s.ring + slot * kSlotBytes;
+    uint8_t* const vb = kb + kSlotBytes / 2;
+    const bool own = p.pos >= blk && p.pos < blk + n;
+    if (own || (n & 15)) {
+      // this step's own key/value row (the QK stage writes it in this launch) from the staged copy,
+      // and zero value rows n..16 KT - 1 (loaded past the chunk: later positions may hold anything,
+      // and P = 0 there must not meet a NaN); the proxy fence orders these generic writes before the
+      // slot's next tensor copy
+      constexpr int CH = HD / 8;                        // 16-byte chunks per row
+      if (own && tid < 2 * CH) {
+        const int jr = p.pos - blk, ch = tid % CH;
+        uint8_t* dst = (tid < CH ? kb : vb) + kv_off(jr, ch, NPS);
+        *reinterpret_cast<uint4*>(dst) = reinterpret_cast<const uint4*>(kvc + (tid < CH ? 0 : HD))[ch];
       }
+      for (int i = tid; i < (16 * KT - n) * CH; i += kConsumerThreads)
+        *reinterpret_cast<uint4*>(vb + kv_off(n + i / CH, i % CH, NPS)) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();
       bar_compute();
     }
-    if (in_group) {
-      for (int base = 0; base < n; base += WPH * PPW) {
-        const int j = base + wi * PPW + sw;
-        const bool valid = j < n;
-        // scores of this sub-warp's position for the warp's heads: packed fp32 FMAs over the
-        // lane's 8 elements, then a sum over the LPP lanes of the position
-        float sc[HW];
-        {
-          const uint4 kw = valid ? *reinterpret_cast<const uint4*>(kb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
-          const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
-          float a[HW];
+    // ---- QK: warps over 8-position tiles ----
+    const int NT = (n + 7) >> 3;
+    float wm = -CUDART_INF_F;
+    const uint32_t kb_a = smem_u32(kb);
+    int* const mx = smax + (si & 1) * kMaxGroup;
+    for (int nt = warp; nt < NT; nt += kConsumerWarps) {
+      // two accumulator chains (even and odd k-steps): half the dependent MMA latency
+      float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+      const int r = nt * 8 + (lane & 7);
+      uint32_t b[KS / 2][4];
 #pragma unroll
-          for (int g = 0; g < HW; ++g) {
-            unsigned long long acc2 = 0ull;
+      for (int kk = 0; kk < KS / 2; ++kk) ldsm_x4(b[kk], kb_a + kv_off(r, 4 * kk + (lane >> 3), NPS));
 #pragma unroll
-            for (int q = 0; q < 4; ++q) ffma2(acc2, bf_lo(kk[q]), bf_hi(kk[q]), qr[g][2 * q], qr[g][2 * q + 1]);
-            a[g] = f2sum(acc2);
+      for (int kk = 0; kk < KS / 2; ++kk) {
+        mma_bf16_16816(d, qa[2 * kk], b[kk][0], b[kk][1]);
+        mma_bf16_16816(e, qa[2 * kk + 1], b[kk][2], b[kk][3]);
+      }
+      const int j0 = nt * 8 + 2 * t4;
+      const float s0 = j0 < n ? (d[0] + e[0]) + (d[2] + e[2]) : -CUDART_INF_F;
+      const float s1 = j0 + 1 < n ? (d[1] + e[1]) + (d[3] + e[3]) : -CUDART_INF_F;
+      if (gid < G) *reinterpret_cast<float2*>(Ssm + gid * NPS + j0) = make_float2(s0, s1);
+      wm = fmaxf(wm, fmaxf(s0, s1));
+    }
+    wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 1));
+    wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 2));
+    if (gid < G && t4 == 0 && warp < NT) atomicMax(mx + gid, max_key(wm));
+    bar_compute();
+    // ---- the new running maxima (every thread, identically) from the slot maxima; the other buffer
+    //      is reset for the next slot ----
+    float Mnew[kMaxGroup], alpha[kMaxGroup];
+    {
+      static_assert(kMaxGroup == 4, "one 16-byte read of the slot maxima");
+      const int4 k4 = *reinterpret_cast<const int4*>(mx);
+      const float ms[kMaxGroup] = {key_max(k4.x), key_max(k4.y), key_max(k4.z), key_max(k4.w)};
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) {
+        Mnew[g] = fmaxf(Mrun[g], ms[g]);
+        alpha[g] = exp2_scale(Mrun[g], Mnew[g]);
+        Mrun[g] = Mnew[g];
+      }
+      if (tid < kMaxGroup) smax[((si + 1) & 1) * kMaxGroup + tid] = max_key(-CUDART_INF_F);
+    }
+    // ---- P = 2^(S - M) as hi/lo bf16 rows of the P tile, two positions per thread ----
+    {
+      const int W2 = 8 * KT;                            // position pairs per head (16 KT positions)
+      for (int e = tid; e < G * W2; e += kConsumerThreads) {
+        const int g = e / W2, j = 2 * (e % W2);
+        const float M = g == 0 ? Mnew[0] : g == 1 ? Mnew[1] : g == 2 ? Mnew[2] : Mnew[3];
+        const float p0 = j < n ? fast_exp2(Ssm[g * NPS + j] - M) : 0.f;
+        const float p1 = j + 1 < n ? fast_exp2(Ssm[g * NPS + j + 1] - M) : 0.f;
+        uint32_t hi, lo;
+        split_bf2(p0, p1, hi, lo);
+        *reinterpret_cast<uint32_t*>(ptile + g * PSTR + j * 2) = hi;
+        *reinterpret_cast<uint32_t*>(ptile + (g + 8) * PSTR + j * 2) = lo;
+      }
+    }
+    bar_compute();
+    // ---- PV ----
+    const float al = gid == 0 ? alpha[0] : gid == 1 ? alpha[1] : gid == 2 ? alpha[2] : gid == 3 ? alpha[3] : 1.f;
+    const uint32_t vb_a = smem_u32(vb);
+#pragma unroll
+    for (int jb = 0; jb < NJ; ++jb) {
+      const int job = warp + jb * kConsumerWarps;
+      if (job < NJOBS) {
+        const int ntile = job % NTO, kpart = job / NTO;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { acc[jb][i] *= al; lacc[jb][i] *= al; }
+        // two position steps per round, their operands loaded first and accumulated in separate
+        // registers (added at the end of the slot): half the dependent MMA latency
+        const int mi = lane >> 3;
+        const uint32_t pa = ptile_a + (((mi & 1) << 3) | (lane & 7)) * PSTR + ((mi >> 1) << 3) * 2;
+        const int vr = 8 * (mi & 1) + (lane & 7);
+        float a2[4] = {0.f, 0.f, 0.f, 0.f}, l2[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int ks = kpart; ks < KT; ks += 2 * KSPLIT) {
+          const bool two = ks + KSPLIT < KT;
+          uint32_t a[4], c[4] = {0u, 0u, 0u, 0u}, b0, b1, b2 = 0u, b3 = 0u;
+          ldsm_x4(a, pa + 32 * ks);
+          ldsm_x2_trans(b0, b1, vb_a + kv_off(16 * ks + vr, ntile, NPS));
+          if (two) {
+            ldsm_x4(c, pa + 32 * (ks + KSPLIT));
+            ldsm_x2_trans(b2, b3, vb_a + kv_off(16 * (ks + KSPLIT) + vr, ntile, NPS));
           }
-          if constexpr (HW == 2) {
-            // both heads in one butterfly: the first exchange leaves head 0's pair sums on the lanes
-            // whose LPP/2 bit is clear and head 1's on the others, the rest reduce within each half
-            const bool up = cl & (LPP / 2);
-            float k = up ? a[1] : a[0];
-            k += __shfl_xor_sync(0xffffffffu, up ? a[0] : a[1], LPP / 2);
-#pragma unroll
-            for (int off = LPP / 4; off >= 1; off >>= 1) k += __shfl_xor_sync(0xffffffffu, k, off);
-            const float other = __shfl_xor_sync(0xffffffffu, k, LPP / 2);
-            sc[0] = up ? other : k;
-            sc[1] = up ? k : other;
-          } else {
-#pragma unroll
-            for (int g = 0; g < HW; ++g) {
-              float k = a[g];
-#pragma unroll
-              for (int off = 1; off < LPP; off <<= 1) k += __shfl_xor_sync(0xffffffffu, k, off);
-              sc[g] = k;
-            }
+          mma_bf16_16816(acc[jb], a, b0, b1);
+          if (ntile == 0) mma_bf16_16816(lacc[jb], a, kOnes, kOnes);
+          if (two) {
+            mma_bf16_16816(a2, c, b2, b3);
+            if (ntile == 0) mma_bf16_16816(l2, c, kOnes, kOnes);
           }
         }
-        // online softmax per sub-warp; o and l are rescaled only in steps where some lane's
-        // maximum rises (warp vote), which after the first positions is rare
-        const uint4 vw = valid ? *reinterpret_cast<const uint4*>(vb + (size_t)j * HD * 2 + cl * 16) : make_uint4(0, 0, 0, 0);
-        const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
 #pragma unroll
-        for (int g = 0; g < HW; ++g) {
-          if (g0 + g < G) {
-            const bool rise = valid && sc[g] > m[g];
-            if (__any_sync(0xffffffffu, rise)) {
-              const float mn = rise ? sc[g] : m[g];
-              const float cr = exp2_scale(m[g], mn);
-              ls[g] *= cr;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) o[g][e] *= cr;
-              m[g] = mn;
-            }
-            const float pe = valid ? fast_exp2(sc[g] - m[g]) : 0.f;
-            ls[g] += pe;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) ffma2_pair(o[g][2 * q], o[g][2 * q + 1], pe, bf_lo(vv[q]), bf_hi(vv[q]));
-          }
-        }
+        for (int i = 0; i < 4; ++i) { acc[jb][i] += a2[i]; lacc[jb][i] += l2[i]; }
       }
     }
     __syncwarp();
@@ -1396,77 +1552,50 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
   }
 
   if (tr && tid == 0) tr[4] = globaltimer();
-  // merge the sub-warps of this warp (lanes with the same piece)
-#pragma unroll
-  for (int g = 0; g < HW; ++g) {
-#pragma unroll
-    for (int off = LPP; off < 32; off <<= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
-      const float lo = __shfl_xor_sync(0xffffffffu, ls[g], off);
-      const float M = fmaxf(m[g], mo);
-      const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
-      ls[g] = ls[g] * fa + lo * fb;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float oo = __shfl_xor_sync(0xffffffffu, o[g][e], off);
-        o[g][e] = o[g][e] * fa + oo * fb;
-      }
-      m[g] = M;
-    }
-  }
-  // every warp's (m, l, o) of its heads into aux, then one thread per (query head, element) folds
-  // the entries of its head group and writes this CTA's partial of that element. When one entry per
-  // warp would not fit aux (4 heads per warp), the upper half of each group's warps first folds into
-  // the lower half through aux (one more barrier), leaving half as many entries.
-  constexpr int stride = HD + 2;
-  constexpr bool two_level = kConsumerWarps * HW * stride * 4 > kAuxBytes;
-  static_assert((kConsumerWarps / 2) * HW * stride * 4 <= kAuxBytes, "attention fold entries fit aux");
-  const int nent = two_level ? WPH / 2 : WPH;   // entries per head group
-  auto put_entry = [&](int slot_idx) {
-    float* ent = s.aux + (size_t)slot_idx * HW * stride;
-#pragma unroll
-    for (int g = 0; g < HW; ++g) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ent[g * stride + cl * 8 + e] = o[g][e];
-      if (cl == 0) { ent[g * stride + HD] = m[g]; ent[g * stride + HD + 1] = ls[g]; }
-    }
-  };
-  if (two_level) {
-    if (in_group && wi >= nent && sw == 0) put_entry(hg * nent + wi - nent);
+  // ---- the chunk's partial: O (unnormalised), M and l per query head ----
+  if constexpr (KSPLIT > 1) {
+    // jobs of the later position residues hand their accumulators to residue 0 through the P tile
+    float* xs = reinterpret_cast<float*>(ptile);
     bar_compute();
-    if (in_group && wi < nent) {
-      const float* ent = s.aux + (size_t)(hg * nent + wi) * HW * stride;
 #pragma unroll
-      for (int g = 0; g < HW; ++g) {
-        const float mo = ent[g * stride + HD], lo = ent[g * stride + HD + 1];
-        const float M = fmaxf(m[g], mo);
-        const float fa = exp2_scale(m[g], M), fb = exp2_scale(mo, M);
-        ls[g] = ls[g] * fa + lo * fb;
+    for (int jb = 0; jb < NJ; ++jb) {
+      const int job = warp + jb * kConsumerWarps;
+      const int ntile = job % NTO, kpart = job / NTO;
+      if (job < NJOBS && kpart > 0) {
+        float* e = xs + (((kpart - 1) * NTO + ntile) * 32 + lane) * 8;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[g][e] = o[g][e] * fa + ent[g * stride + cl * 8 + e] * fb;
-        m[g] = M;
+        for (int i = 0; i < 4; ++i) { e[i] = acc[jb][i]; e[4 + i] = lacc[jb][i]; }
       }
     }
     bar_compute();
-  }
-  if (in_group && wi < nent && sw == 0) put_entry(hg * nent + wi);
-  bar_compute();
-  for (int idx = tid; idx < G * HD; idx += kConsumerThreads) {
-    const int g = idx / HD, e = idx % HD;
-    const float* ent = s.aux + (size_t)(g / HW) * nent * HW * stride + (g % HW) * stride;
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < nent; ++w) M = fmaxf(M, ent[w * HW * stride + HD]);
-    float L = 0.f, acc = 0.f;
-    for (int w = 0; w < nent; ++w) {
-      const float* ew = ent + w * HW * stride;
-      const float wt = exp2_scale(ew[HD], M);
-      L = fmaf(ew[HD + 1], wt, L);
-      acc = fmaf(ew[e], wt, acc);
+#pragma unroll
+    for (int jb = 0; jb < NJ; ++jb) {
+      const int job = warp + jb * kConsumerWarps;
+      const int ntile = job % NTO, kpart = job / NTO;
+      if (job < NJOBS && kpart == 0) {
+        for (int k = 1; k < KSPLIT; ++k) {
+          const float* e = xs + (((k - 1) * NTO + ntile) * 32 + lane) * 8;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { acc[jb][i] += e[i]; lacc[jb][i] += e[4 + i]; }
+        }
+      }
     }
-    uint64_t* dg = p.attn_part + (((size_t)h * G + g) * p.kv_chunks_max + c) * stride;
+  }
+  {
     const uint32_t tg = tag_of(p.tag_epoch, l);
-    st_pair(dg + e, acc, tg);
-    if (e == 0) st_pair2(dg + HD, M, L, tg);   // (hd + 2) even: 16-byte aligned
+#pragma unroll
+    for (int jb = 0; jb < NJ; ++jb) {
+      const int job = warp + jb * kConsumerWarps;
+      const int ntile = job % NTO, kpart = job / NTO;
+      if (job < NJOBS && kpart == 0 && gid < G) {
+        uint64_t* dg = p.attn_part + (((size_t)h * G + gid) * p.kv_chunks_max + c) * (HD + 2);
+        st_pair2(dg + ntile * 8 + 2 * t4, acc[jb][0] + acc[jb][2], acc[jb][1] + acc[jb][3], tg);
+        if (ntile == 0 && t4 == 0) {
+          const float M = gid == 0 ? Mrun[0] : gid == 1 ? Mrun[1] : gid == 2 ? Mrun[2] : Mrun[3];
+          st_pair2(dg + HD, M, lacc[jb][0] + lacc[jb][2], tg);   // (hd + 2) even: 16-byte aligned
+        }
+      }
+    }
   }
   if (tr && tid == 0) tr[5] = globaltimer();
   if (!p.sync) return it;
@@ -1552,6 +1681,7 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
     if (tr && tid == 0) {
       tr[0] = ((unsigned long long)t.op << 32) | (unsigned long long)t.layer << 16 | (unsigned)ti;
       tr[1] = tr[2] = globaltimer();
+      tr[13] = clock64();
     }
     if (is_gemv(t.op)) {
       const GemvGeom& g = p.geom[gemv_slot_of(t.op)];
@@ -1621,7 +1751,10 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
     } else if (t.op == OP_ARGMAX) {
       grid_argmax(p);
     }
-    if (tr && tid == 0) tr[3] = globaltimer();
+    if (tr && tid == 0) {
+      tr[3] = globaltimer();
+      tr[14] = clock64();
+    }
   }
 }
 

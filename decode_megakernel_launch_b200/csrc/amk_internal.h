@@ -7,6 +7,7 @@
 //   per layer l:  QKV(l) -> ATTN(l) -> O(l) -> GU(l) -> DOWN(l);   then LM (head + argmax).
 // Every GEMV stage is row-split over all CTAs; ATTN is split over (KV head, KV chunk).
 #pragma once
+#include <cuda.h>       // CUtensorMap (the descriptors are encoded through the runtime's driver entry point)
 #include <stdint.h>
 
 #include "../../include/amk.h"
@@ -44,15 +45,20 @@ constexpr int kThreads         = kConsumerThreads + 32;    // + 1 producer (bulk
 constexpr int kSlotBytes       = AMK_SLOT_BYTES;           // one bulk-copy ring slot
 constexpr int kSlots           = AMK_SLOTS;                // ring depth
 constexpr int kInflight        = AMK_INFLIGHT;             // outstanding copies, <= kSlots
-// While the compute warps hold a landed slot longer than kStallNs (they wait on a counter), the
-// producer warms L2 with up to kPfItems upcoming ring items, one per kPfGapNs (a little faster than
-// one SM's share of HBM bandwidth), so HBM keeps streaming through the stage transition; 10 items
-// of 64 KB on 148 SMs use at most 97 MB of the 126 MB L2. kPfItems = 0 disables it.
+// The producer warms L2 with up to kPfItems upcoming ring items, one per kPfGapNs (a little faster
+// than one SM's share of HBM bandwidth: 64 KB per 1.2 us on 148 SMs is 7.9 TB/s; at 0.8 us the
+// queues it builds slow every other load), so HBM keeps streaming through the stage transitions:
+// while the compute warps hold a landed slot longer than kStallNs (they wait on a counter) and,
+// with kPfContinuous, between stalls too. 10 items of 64 KB on 148 SMs use at most 97 MB of the
+// 126 MB L2. kPfItems = 0 disables it.
 #ifndef AMK_PF_ITEMS
 #define AMK_PF_ITEMS 10
 #endif
 #ifndef AMK_PF_GAP_NS
-#define AMK_PF_GAP_NS 800
+#define AMK_PF_GAP_NS 1200
+#endif
+#ifndef AMK_PF_CONTINUOUS
+#define AMK_PF_CONTINUOUS 1
 #endif
 #ifndef AMK_PF_STALL_NS
 #define AMK_PF_STALL_NS 200
@@ -60,6 +66,7 @@ constexpr int kInflight        = AMK_INFLIGHT;             // outstanding copies
 constexpr int kPfItems = AMK_PF_ITEMS;
 constexpr unsigned kPfGapNs = AMK_PF_GAP_NS;
 constexpr unsigned kStallNs = AMK_PF_STALL_NS;
+constexpr bool kPfContinuous = AMK_PF_CONTINUOUS != 0;
 static_assert(kInflight >= 1 && kInflight <= kSlots, "ring in-flight bound");
 static_assert(kSlotBytes % 256 == 0 && kSlotBytes >= 32768, "ring slot holds a 32 KB weight row");
 constexpr int kRowBlock        = 128;                      // GEMV rows per epilogue block
@@ -196,6 +203,9 @@ struct Params {
   const uint16_t* lm_s;        // scales or null
   uint16_t* kcache;            // bf16 [L][Hkv][max_seq][hd]
   uint16_t* vcache;
+  // the caches as 2-D [L Hkv max_seq][hd] bf16 tensors with 128-byte swizzle: [0] boxes of 64
+  // columns x 64 rows, [1] of 64 columns x 16 rows (for the last rows of a chunk)
+  CUtensorMap kmap[2], vmap[2];
   const float* rope;           // interleaved (cos, sin) [max_seq][hd/2][2]
   // scratch (device)
   // tagged words (see tag_of)
@@ -230,6 +240,10 @@ struct Params {
   int*   next_token;
   int sync;                    // 1 = persistent megakernel (waits/signals), 0 = op-per-kernel
 };
+
+// Encodes p.kmap and p.vmap from p.kcache, p.vcache and the dims in p (host). Returns AMK_OK or
+// AMK_ERR_CUDA when the driver's encoder is unavailable or refuses the layout.
+int encode_kv_maps(Params& p);
 
 // ---- shared host/device helpers ----------------------------------------------------------------
 AMK_HD inline int packed_row_source(int role, int hd, int ffn, int packed_row) {

@@ -198,6 +198,7 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
     p.lm_s = (!d.tied_head && i8) ? static_cast<const uint16_t*>(w->slm) : nullptr;
     p.kcache = static_cast<uint16_t*>(w->k_cache);
     p.vcache = static_cast<uint16_t*>(w->v_cache);
+    if (encode_kv_maps(p) != AMK_OK) return AMK_ERR_CUDA;
     p.rope = reinterpret_cast<const float*>(B + o_rope);
     p.x = reinterpret_cast<uint64_t*>(B + o_x);
     p.xres = reinterpret_cast<float*>(B + o_xres);

@@ -171,7 +171,8 @@ int  amk_decode_step_unfused(amk_handle* h, int token_id, int pos, float* logits
 /* Sticky device status without synchronizing: AMK_OK or AMK_ERR_DEVICE_TIMEOUT (a wait expired in
  * an earlier launch). `detail` (may be NULL) receives the raw status word: bits 0..15 the counter
  * or slot index that expired, bits 16..23 the wait kind (1 counter, 2 full slot, 3 empty slot,
- * 4 next-token id out of range at launch, 5 producer waiting for its own copy to land). */
+ * 4 next-token id out of range at launch, 5 producer waiting for its own copy to land, 6 a tagged
+ * input that never became current, 7 shared memory not 1024-byte aligned for the swizzled KV copies). */
 int  amk_status(const amk_handle* h, uint32_t* detail);
 
 /* Last CUDA error string seen by this library on this thread ("" if none). */
@@ -239,10 +240,12 @@ int amk_plan_check(const amk_dims* dims, int grid, int mutation, char* msg, int 
  *   GEMV:      [4] inputs loaded and quantised, [5] first ring slot landed, [6] thread 0's last row
  *              computed, [10] every warp's last row computed, [11] last result block's bulk store
  *              issued, [7] signal issued (after that store completed);
- *   attention: [4] KV chunk done, [5] partial issued, [6] ticket taken, [7] head merged and signalled
- *              (0 unless this chunk merged the head);
+ *   attention: [10] q, k, v staged, [11] first KV slot landed, [4] KV chunk done, [5] partial
+ *              issued, [6] ticket taken, [7] head merged and signalled (0 unless this chunk merged
+ *              the head; records are not cleared between steps, so compare [7] with [6]);
  *   producer:  [8] the task's first ring item issued, [9] its last item issued;
- *   GEMV inputs: [12] thread 0's input words landed.
+ *   GEMV inputs: [12] thread 0's input words landed;
+ *   every task: [13] and [14] the SM's clock64 at [1] and [3] (so the SM clock during the task).
  * Copies up to `max_records` records into the host buffer `out` (synchronizes the device) and
  * returns how many were written, or a negative code. Record r of CTA b is at index
  * b * (max tasks per CTA) + r; unused records and stamps are zero. The task word holds
