@@ -640,8 +640,10 @@ def _kernel_hash():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=8)
+    # defaults: 200 timed launches (8 warm-up) for the kernel; the reference arm (the CPU oracle, ~3 s
+    # per full-depth 8B step) defaults to 20 (3 warm-up), so its run ends within a few minutes
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", default="amk", choices=["amk", "reference"])
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -651,6 +653,10 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (smaller cases for profiler captures; not a bench line)")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else 200
+    if args.warmup is None:
+        args.warmup = 3 if args.impl == "reference" else 8
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from decode_megakernel_launch_b200 import synth

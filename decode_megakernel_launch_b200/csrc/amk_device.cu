@@ -1356,14 +1356,21 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
   if (p.sync && t.wait_ctr >= 0) wait_counter(p, t.wait_ctr, t.wait_mult);
   if (tr && tid == 0) tr[2] = globaltimer();
 
-  // queries of this KV head's group, pre-scaled by log2(e) / sqrt(hd), and this position's key and
-  // value rows (bf16), staged in shared memory (the GEMV partial-sum region, which attention tasks
-  // do not use) in one round trip. The QKV stage publishes them in packed row order: packed row j
-  // of a head is element j / 2 (j even) or hd/2 + j / 2 (j odd).
+  // queries of this KV head's group, pre-scaled by log2(e) / sqrt(hd), as the A operand of the QK
+  // MMAs (q tile: bf16 rows 0..G-1 the heads, rows 8..8+G-1 what rounding left over, other rows
+  // zero), and this position's key and value rows (bf16), staged in shared memory (the GEMV
+  // partial-sum region, which attention tasks do not use) in one round trip. The QKV stage publishes
+  // them in packed row order: packed row j of a head is element j / 2 (j even) or hd/2 + j / 2 (j odd).
   const float qs = 1.4426950408889634f * rsqrtf((float)HD);
-  float* qsm = s.part;
-  uint16_t* kvc = reinterpret_cast<uint16_t*>(s.part + kMaxGroup * 128);   // [HD] k, then [HD] v
+  constexpr int QSTR = HD * 2 + 16;                    // q tile row bytes (padded: conflict-free ldmatrix)
+  uint8_t* const qtile = reinterpret_cast<uint8_t*>(s.part);
+  uint16_t* kvc = reinterpret_cast<uint16_t*>(qtile + 16 * QSTR);   // [HD] k, then [HD] v
+  static_assert(16 * QSTR + 4 * HD <= kPartBytes, "q tile and this position's k, v fit the partial region");
   auto unpack = [](int j) { return (j & 1) ? (j >> 1) + HD / 2 : (j >> 1); };
+  for (int i = tid; i < 16 * QSTR / 16; i += kConsumerThreads) {   // rows past the group stay zero
+    const int row = (i * 16) / QSTR;
+    if ((row & 7) >= G) reinterpret_cast<uint4*>(qtile)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
   {
     // up to two tagged pairs of q and (the first 2 * HD threads) one of k or v per thread, all in
     // one batch (G * HD <= 512)
@@ -1381,7 +1388,14 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int iq = tid + j * kConsumerThreads;
-      if (iq < G * HD) qsm[(iq / HD) * HD + unpack(iq % HD)] = __uint_as_float(v[j].x) * qs;
+      if (iq < G * HD) {
+        const float x = __uint_as_float(v[j].x) * qs;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+        const int g = iq / HD, e = unpack(iq % HD);
+        *reinterpret_cast<__nv_bfloat16*>(qtile + g * QSTR + 2 * e) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(qtile + (g + 8) * QSTR + 2 * e) = lo;
+      }
     }
     if (ik < 2 * HD) kvc[(ik < HD ? 0 : HD) + unpack(ik % HD)] = f2bf(__uint_as_float(v[2].x));
   }
@@ -1396,20 +1410,12 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
   bar_compute();
   if (tr && tid == 0) tr[10] = globaltimer();
 
-  // q as the A operand (see above): fragments for the whole task
   constexpr int KS = HD / 16;                          // k-steps of the QK contraction
   const int gid = lane >> 2, t4 = lane & 3;
-  uint32_t qa[KS][4];
-#pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-    if (gid < G) {
-      const float* qq = qsm + gid * HD + 16 * ks + 2 * t4;
-      x0 = qq[0]; x1 = qq[1]; x2 = qq[8]; x3 = qq[9];
-    }
-    split_bf2(x0, x1, qa[ks][0], qa[ks][1]);
-    split_bf2(x2, x3, qa[ks][2], qa[ks][3]);
-  }
+  // this lane's row address in the q and P tiles for ldmatrix.x4 of an A operand (tile i of the four:
+  // rows 8 (i & 1).., columns 8 (i >> 1).. of the 16-column step)
+  const int arow = (((lane >> 3) & 1) << 3) | (lane & 7), acol = ((lane >> 4) & 1) << 3;
+  const uint32_t qa_a = smem_u32(qtile) + arow * QSTR + acol * 2;
 
   // PV jobs: (output tile of 8 dimensions, position-step residue); most configurations give one
   // job per warp
@@ -1459,23 +1465,29 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
     float wm = -CUDART_INF_F;
     const uint32_t kb_a = smem_u32(kb);
     int* const mx = smax + (si & 1) * kMaxGroup;
-    for (int nt = warp; nt < NT; nt += kConsumerWarps) {
-      // two accumulator chains (even and odd k-steps): half the dependent MMA latency
-      float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
-      const int r = nt * 8 + (lane & 7);
-      uint32_t b[KS / 2][4];
+    if (warp < NT) {
+      // the q fragments, for this slot's tiles of the warp (not held across the slot: registers)
+      uint32_t qf[KS][4];
 #pragma unroll
-      for (int kk = 0; kk < KS / 2; ++kk) ldsm_x4(b[kk], kb_a + kv_off(r, 4 * kk + (lane >> 3), NPS));
+      for (int ks = 0; ks < KS; ++ks) ldsm_x4(qf[ks], qa_a + 32 * ks);
+      for (int nt = warp; nt < NT; nt += kConsumerWarps) {
+        // two accumulator chains (even and odd k-steps): half the dependent MMA latency
+        float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+        const int r = nt * 8 + (lane & 7);
+        uint32_t b[KS / 2][4];
 #pragma unroll
-      for (int kk = 0; kk < KS / 2; ++kk) {
-        mma_bf16_16816(d, qa[2 * kk], b[kk][0], b[kk][1]);
-        mma_bf16_16816(e, qa[2 * kk + 1], b[kk][2], b[kk][3]);
+        for (int kk = 0; kk < KS / 2; ++kk) ldsm_x4(b[kk], kb_a + kv_off(r, 4 * kk + (lane >> 3), NPS));
+#pragma unroll
+        for (int kk = 0; kk < KS / 2; ++kk) {
+          mma_bf16_16816(d, qf[2 * kk], b[kk][0], b[kk][1]);
+          mma_bf16_16816(e, qf[2 * kk + 1], b[kk][2], b[kk][3]);
+        }
+        const int j0 = nt * 8 + 2 * t4;
+        const float s0 = j0 < n ? (d[0] + e[0]) + (d[2] + e[2]) : -CUDART_INF_F;
+        const float s1 = j0 + 1 < n ? (d[1] + e[1]) + (d[3] + e[3]) : -CUDART_INF_F;
+        if (gid < G) *reinterpret_cast<float2*>(Ssm + gid * NPS + j0) = make_float2(s0, s1);
+        wm = fmaxf(wm, fmaxf(s0, s1));
       }
-      const int j0 = nt * 8 + 2 * t4;
-      const float s0 = j0 < n ? (d[0] + e[0]) + (d[2] + e[2]) : -CUDART_INF_F;
-      const float s1 = j0 + 1 < n ? (d[1] + e[1]) + (d[3] + e[3]) : -CUDART_INF_F;
-      if (gid < G) *reinterpret_cast<float2*>(Ssm + gid * NPS + j0) = make_float2(s0, s1);
-      wm = fmaxf(wm, fmaxf(s0, s1));
     }
     wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 1));
     wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 2));
@@ -1523,9 +1535,8 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
         for (int i = 0; i < 4; ++i) { acc[jb][i] *= al; lacc[jb][i] *= al; }
         // two position steps per round, their operands loaded first and accumulated in separate
         // registers (added at the end of the slot): half the dependent MMA latency
-        const int mi = lane >> 3;
-        const uint32_t pa = ptile_a + (((mi & 1) << 3) | (lane & 7)) * PSTR + ((mi >> 1) << 3) * 2;
-        const int vr = 8 * (mi & 1) + (lane & 7);
+        const uint32_t pa = ptile_a + arow * PSTR + acol * 2;
+        const int vr = arow;   // ldmatrix.x2.trans: lanes 0..15 give rows 0..15 of the position step
         float a2[4] = {0.f, 0.f, 0.f, 0.f}, l2[4] = {0.f, 0.f, 0.f, 0.f};
         for (int ks = kpart; ks < KT; ks += 2 * KSPLIT) {
           const bool two = ks + KSPLIT < KT;
