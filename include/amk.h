@@ -96,7 +96,10 @@ typedef struct amk_weights {
   void*              v_cache;     /* bf16 [L][Hkv][max_seq][hd], read and written            */
 } amk_weights;
 
-/* Optional tuning and test knobs; pass NULL to amk_create for the defaults (all fields 0). */
+/* Optional tuning and test knobs; pass NULL to amk_create for the defaults (all fields 0). This
+ * fourth argument of amk_create is an addition of this library: it carries what the pages' schedule
+ * search tunes (skill page, "The ScheduleConfig knobs": tiling.attention.kv_block, SM assignment)
+ * plus the wait limit, tracing and one failure-injection hook for tests. */
 typedef struct amk_options {
   int grid;              /* persistent CTAs; 0 = one per SM                                    */
   int kv_block;          /* minimum positions per attention chunk; 0 = 64                      */
@@ -111,7 +114,9 @@ typedef struct amk_handle amk_handle;
 
 /* ---- packing --------------------------------------------------------------------------------- */
 
-/* Bytes of the packed weight buffer for `rows` x `cols` in `dst_dtype` (rows * cols * 1 for int8,
+/* Implements the storage of the quantized weight-only variants (technical summary, "Key
+ * Contributions", Quantized Megakernels: int8 and int4 weight-only kernels).
+ * Bytes of the packed weight buffer for `rows` x `cols` in `dst_dtype` (rows * cols * 1 for int8,
  * * 2 for bf16, / 2 for int4; int4 needs an even `cols`, else 0). */
 size_t amk_packed_bytes(int rows, int cols, int dst_dtype);
 
@@ -121,7 +126,9 @@ size_t amk_packed_bytes(int rows, int cols, int dst_dtype);
  * hold gate row i (source row i) and up row i (source row ffn + i). */
 int amk_packed_row_source(int role, const amk_dims* dims, int rows, int packed_row);
 
-/* Device-side weight packer (W8A16 / W4A16 quantiser, bf16 copier).
+/* Device-side weight packer (W8A16 / W4A16 quantiser, bf16 copier). Implements the int8 (W8A16)
+ * and int4 weight-only quantisation the abstract and the technical summary ("Key Contributions",
+ * Quantized Megakernels) name; the per-row symmetric scheme is this library's reading of them.
  *   src:        device, [rows, cols] row-major in `src_dtype`; for QKV the rows of Wq, Wk, Wv
  *               stacked, for GATE_UP the rows of Wgate then Wup.
  *   packed_out: device, amk_packed_bytes(rows, cols, dst_dtype) bytes, rows in the role's order.
@@ -138,20 +145,27 @@ int amk_pack_weight(int role, const amk_dims* dims, const void* src, int src_dty
 
 /* ---- handle lifetime ------------------------------------------------------------------------- */
 
-/* Validates dims/pointers, builds and statically checks the per-CTA task list, allocates the
+/* Implements the technical summary's "Methodology", Layer 0 (one persistent block per SM walking a
+ * task order with wait -> dispatch -> signal on monotonic counters) and its safety gate (the task
+ * list is checked for satisfiable waits, stage order and producer counts before any launch).
+ * Validates dims/pointers, builds and statically checks the per-CTA task list, allocates the
  * handle's device state and checks that the persistent grid is co-resident. Synchronous.
  * Supported: head_dim in {64,128}; Hq/Hkv in 1..4; d_model, ffn and Hq*hd multiples of 64 and
  * at most 16384; weight rows of at most 32 KB. On failure *out is NULL. */
 int  amk_create(const amk_dims* dims, const amk_weights* weights, const amk_options* options,
                 amk_handle** out);
 
-/* Frees the handle's own device and host state (never the caller's buffers). Synchronizes the
+/* Lifetime call of this library (the pages print no API).
+ * Frees the handle's own device and host state (never the caller's buffers). Synchronizes the
  * device first. NULL is ignored. */
 void amk_destroy(amk_handle* h);
 
 /* ---- the decode step ------------------------------------------------------------------------- */
 
-/* One greedy decode step in ONE persistent launch on `stream`.
+/* Implements the technical summary's "Problem Statement" (single-stream autoregressive decoding at
+ * batch size 1, floor = weight bytes / HBM bandwidth) as the abstract describes it: the whole
+ * forward pass of one token in ONE persistent launch, greedy.
+ * One greedy decode step in ONE persistent launch on `stream`.
  *   token_id:       token at position `pos`, in [0, V); or -1 to read it from *next_token_out
  *                   (written by the previous step on the same stream: device-side feedback).
  *   pos:            absolute position, 0 <= pos < max_seq. K/V are written at `pos` and attention
@@ -162,13 +176,17 @@ void amk_destroy(amk_handle* h);
 int  amk_decode_step(amk_handle* h, int token_id, int pos, float* logits_out, int* next_token_out,
                      void* stream);
 
-/* Ablation: the same step with the same device routines, launched one kernel per operation
+/* The conventional execution the technical summary's "Problem Statement" contrasts with (a separate
+ * kernel per operator), kept as an ablation.
+ * Ablation: the same step with the same device routines, launched one kernel per operation
  * (per layer: QKV, attention partials, attention merge, O, gate/up, down; then LM head and the
  * argmax), so activations cross HBM between kernels and there is no cross-SM counter. */
 int  amk_decode_step_unfused(amk_handle* h, int token_id, int pos, float* logits_out,
                              int* next_token_out, void* stream);
 
-/* Sticky device status without synchronizing: AMK_OK or AMK_ERR_DEVICE_TIMEOUT (a wait expired in
+/* The pages' rule that an unsafe schedule ends in a clean rejection, never a hung GPU (skill page,
+ * "HARD HONESTY RULES"), carried to run time: every device wait is bounded and reports here.
+ * Sticky device status without synchronizing: AMK_OK or AMK_ERR_DEVICE_TIMEOUT (a wait expired in
  * an earlier launch). `detail` (may be NULL) receives the raw status word: bits 0..15 the counter
  * or slot index that expired, bits 16..23 the wait kind (1 counter, 2 full slot, 3 empty slot,
  * 4 next-token id out of range at launch, 5 producer waiting for its own copy to land, 6 a tagged
@@ -221,11 +239,16 @@ typedef struct amk_plan_info {
 
 int amk_plan_info_get(const amk_handle* h, amk_plan_info* out);
 
-/* Bytes one decode step at `pos` must read: weights (+scales), one embedding row, the norm
+/* The numerator of the technical summary's floor t_min = weight_bytes / HBM_bandwidth ("Problem
+ * Statement"), plus the KV bytes a step reads.
+ * Bytes one decode step at `pos` must read: weights (+scales), one embedding row, the norm
  * gains and the KV cache over positions 0..pos of every layer. Host-only, no GPU. */
 uint64_t amk_step_bytes(const amk_dims* dims, int pos);
 
-/* Static task-list check without a GPU: builds the plan for `dims` on `grid` CTAs, optionally
+/* The safety gate of the technical summary's "Methodology" (deadlock-freedom: satisfiable wait
+ * thresholds 1 <= t <= #producers and valid per-SM orders; race-freedom: every producer of a counter
+ * in an earlier stage; reachability), run without a GPU.
+ * Static task-list check without a GPU: builds the plan for `dims` on `grid` CTAs, optionally
  * plants one defect (mutation 0 = none; 1 drop a signal, 2 raise a wait threshold above its
  * producer count, 3 swap two tasks of one CTA against stage order, 4 make a wait refer to a
  * later stage, 5 drop a stage's producer), runs the checker and writes its verdict to `msg`.
@@ -234,7 +257,9 @@ int amk_plan_check(const amk_dims* dims, int grid, int mutation, char* msg, int 
 
 /* ---- tracing --------------------------------------------------------------------------------- */
 
-/* With options.trace = 1, every CTA records AMK_TRACE_WORDS uint64 per task of the last step:
+/* The localisation of the cross-SM synchronisation cost the technical summary's "Experimental
+ * Results" (Diagnosis) reports, as per-task timestamps.
+ * With options.trace = 1, every CTA records AMK_TRACE_WORDS uint64 per task of the last step:
  *   [0] task word, [1] start, [2] inputs may be read (its counter seen), [3] done, and
  *   %globaltimer stamps (ns) of its phases:
  *   GEMV:      [4] inputs loaded and quantised, [5] first ring slot landed, [6] thread 0's last row
