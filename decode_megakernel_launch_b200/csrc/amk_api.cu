@@ -292,6 +292,7 @@ int amk_create(const amk_dims* dims, const amk_weights* w, const amk_options* op
   for (int i = 0; i < 5; ++i) p.geom[i] = pl.geom[i];
   p.kv_block = h->opt.kv_block > 0 ? h->opt.kv_block : 64;
   p.kv_chunks_max = pl.kv_chunks_max;
+  p.kv_chunks_short = pl.kv_chunks_short;
   p.timeout_ns = (unsigned long long)(h->opt.timeout_ms > 0 ? h->opt.timeout_ms : 2000) * 1000000ull;
   p.max_tasks_per_cta = h->max_tasks_per_cta;
 

@@ -379,7 +379,7 @@ __device__ __forceinline__ void task_range(const Params& p, const Task& t, int& 
   begin = end = 0;
   if (t.op == OP_ATTN) {
     const int P = p.pos + 1;
-    const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
+    const int C = attn_num_chunks(P, p.kv_block, attn_chunk_cap(P, p.kv_chunks_max, p.kv_chunks_short));
     if (t.b < C) attn_chunk_range(P, C, t.b, &begin, &end);
   } else if (is_gemv(t.op)) {
     end = t.b;
@@ -1348,7 +1348,7 @@ uint32_t attn_task(const Params& p, const Task t, uint32_t it, unsigned long lon
   const int G = p.Hq / p.Hkv;
   const int h = t.a, c = t.b, l = t.layer;
   const int P = p.pos + 1;
-  const int C = attn_num_chunks(P, p.kv_block, p.kv_chunks_max);
+  const int C = attn_num_chunks(P, p.kv_block, attn_chunk_cap(P, p.kv_chunks_max, p.kv_chunks_short));
   if (c >= C) return it;
   int cb, ce;
   attn_chunk_range(P, C, c, &cb, &ce);
@@ -1756,7 +1756,7 @@ __device__ void compute(const Params& p, const Task* tasks, int nt) {
       if (p.hd == 64) it = attn_task<64>(p, t, it, tr);
       else it = attn_task<128>(p, t, it, tr);
     } else if (t.op == OP_MERGE) {
-      const int C = attn_num_chunks(p.pos + 1, p.kv_block, p.kv_chunks_max);
+      const int C = attn_num_chunks(p.pos + 1, p.kv_block, attn_chunk_cap(p.pos + 1, p.kv_chunks_max, p.kv_chunks_short));
       if (p.hd == 64) merge_head<64>(p, t.a, C, t.layer);
       else merge_head<128>(p, t.a, C, t.layer);
     } else if (t.op == OP_ARGMAX) {

@@ -229,7 +229,8 @@ struct Params {
   const int*  task_off;        // [grid + 1]
   GemvGeom geom[5];            // QKV, O, GU, DOWN, LM
   int kv_block;
-  int kv_chunks_max;
+  int kv_chunks_max;           // attention chunks per KV head at most (the plan's tasks, partial rows)
+  int kv_chunks_short;         // the cap below kLongContext positions
   unsigned long long timeout_ns;
   // per launch
   uint32_t epoch;              // counter targets are epoch * producers
@@ -257,6 +258,12 @@ AMK_HD inline int packed_row_source(int role, int hd, int ffn, int packed_row) {
 
 // Attention chunking of positions 0..P-1 of one KV head: chunks of cs = ceil(P / c) positions,
 // c = min(cmax, ceil(P / kv_block)); the count returned is ceil(P / cs), so no chunk is empty.
+// Chunk cap for P positions: below kLongContext the merge's one 16-chunk batch (one L2 round trip)
+// beats spreading a short cache over every CTA; from there on each chunk streams several ring slots
+// and more CTAs pay more (1B-shaped, 32K positions: 16 chunks 0.930 ms, 18 chunks 0.913 ms per step;
+// 8B-shaped, 1K: 16 chunks 1.850 ms, 18 chunks 1.877 ms).
+constexpr int kLongContext = 4096;
+AMK_HD inline int attn_chunk_cap(int P, int cmax, int cshort) { return P >= kLongContext ? cmax : cshort; }
 AMK_HD inline int attn_num_chunks(int P, int kv_block, int cmax) {
   if (P < 1) return 1;
   int c = (P + kv_block - 1) / kv_block;

@@ -219,6 +219,7 @@ extern "C" int amk_decode_step_noalloc(const amk_dims* dims, const amk_weights* 
     for (int i = 0; i < 5; ++i) p.geom[i] = pl.geom[i];
     p.kv_block = 64;
     p.kv_chunks_max = pl.kv_chunks_max;
+    p.kv_chunks_short = pl.kv_chunks_short;
     p.timeout_ns = 2000ull * 1000000ull;
     S.zero_off = zero_begin;
     S.zero_bytes = total - zero_begin;

@@ -139,9 +139,10 @@ int build_plan(const amk_dims& d, int grid, int kv_chunks_max, Plan* out, std::s
   // attention chunks per KV head; the (head, chunk) tasks go round-robin over the CTAs, so a grid
   // smaller than Hkv gives some CTAs several heads
   // at most 16 chunks per KV head by default: the merge then gathers them in one round trip
-  int cmax = kv_chunks_max > 0 ? kv_chunks_max : std::min(grid / Hkv, 16);
+  int cmax = kv_chunks_max > 0 ? kv_chunks_max : std::min(grid / Hkv, 32);
   if (cmax < 1) cmax = 1;
   p.kv_chunks_max = cmax;
+  p.kv_chunks_short = kv_chunks_max > 0 ? kv_chunks_max : std::min(grid / Hkv, 16);
   p.n_counters = L * CTR_PER_LAYER;
   const int wk = d.weight_dtype;
   make_geom(d.d_model, wk, &p.geom[0]);                           // QKV: K = d

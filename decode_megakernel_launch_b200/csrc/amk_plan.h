@@ -16,6 +16,7 @@ struct StageList {            // one launch of the op-per-kernel ablation
 struct Plan {
   int grid = 0;
   int kv_chunks_max = 0;
+  int kv_chunks_short = 0;
   int n_counters = 0;
   GemvGeom geom[5];
   std::vector<Task> tasks;        // persistent kernel: all CTAs' lists back to back

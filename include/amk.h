@@ -103,7 +103,8 @@ typedef struct amk_weights {
 typedef struct amk_options {
   int grid;              /* persistent CTAs; 0 = one per SM                                    */
   int kv_block;          /* minimum positions per attention chunk; 0 = 64                      */
-  int max_kv_chunks;     /* cap on attention chunks per KV head; 0 = min(grid / Hkv, 16)       */
+  int max_kv_chunks;     /* cap on attention chunks per KV head; 0 = min(grid / Hkv, 16) below
+                            4096 positions, min(grid / Hkv, 32) from 4096 on                    */
   int timeout_ms;        /* bound on every device wait; 0 = 2000 ms                            */
   int trace;             /* 1: record per-task timestamps (see amk_trace_read)                 */
   int test_drop_signal;  /* TEST ONLY: 1 + index of a counter signal the planner omits, so the
