@@ -630,10 +630,16 @@ def _dram_traffic(workload, algorithmic_bytes):
 
 
 def _kernel_hash():
+    """Hash of the kernel sources with comments and blank space removed, so that a comment edit does
+    not disown counters taken on the same code."""
     import hashlib
+    import re
     h = hashlib.sha1()
     for f in sorted(os.listdir(os.path.join(ROOT, "decode_megakernel_launch_b200", "csrc"))):
-        h.update(open(os.path.join(ROOT, "decode_megakernel_launch_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "decode_megakernel_launch_b200", "csrc", f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(f.encode() + b"\0" + " ".join(text.split()).encode())
     return h.hexdigest()[:12]
 
 

@@ -1,9 +1,10 @@
 // Device code of libamk (sm_100a): the persistent decode kernel, its routines, and the weight packer.
 //
 // One CTA per SM, compute warps + 1: the last warp is the producer, whose elected lane streams every byte this CTA
-// will read (weight rows of its GEMV tasks, KV rows of its attention chunk) into a kSlots x kSlotBytes
-// shared-memory ring with cp.async.bulk, completion tracked by one mbarrier per slot; at most
-// kInflight copies are outstanding at once. The producer
+// will read into a kSlots x kSlotBytes shared-memory ring: weight rows of its GEMV tasks with
+// cp.async.bulk, the keys and values of its attention chunk as 128-byte-swizzled tensor boxes with
+// cp.async.bulk.tensor; completion is tracked by one mbarrier per slot and at most kInflight copies
+// are outstanding at once, while the same lane warms L2 with the items that follow. The producer
 // never waits on other CTAs, so the next tasks' weights arrive while the compute warps wait on a
 // counter: this is the "prefetch the next layer's weights while the current layer computes" of
 // "AutoMegaKernel: A Statically-Checked Agent Harness for Self-Retargeting Megakernel Synthesis"
@@ -683,11 +684,7 @@ __device__ __forceinline__ int dp2a_hi_su(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
-// Vector loads of N consecutive elements (N in {2, 4, 8, 16}) into fp32 registers.
-// Vector loads of N consecutive elements of a vector written earlier in this launch by other CTAs.
-// They may allocate in L1 (the row partitions of a CTA read the same elements, and L1 merges those
-// requests): every such read follows, in this CTA, an acquire on the counter of the stage that wrote
-// the vector plus a CTA barrier, so by the memory model it observes the released values.
+// Vector loads of N consecutive fp32 elements (N in {2, 4, 8, 16}) through L1.
 template <int N>
 __device__ __forceinline__ void ld_f32_ca(const float* p, float* o) {
   if constexpr (N >= 4) {
