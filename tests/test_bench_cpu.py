@@ -43,3 +43,30 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"]
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    # the DRAM-traffic ratio stays attached to counters taken on the same code: a comment edit keeps
+    # the hash, a code edit changes it
+    import shutil
+    src = os.path.join(ROOT, "decode_megakernel_launch_b200", "csrc")
+    dst = tmp_path / "decode_megakernel_launch_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench._kernel_hash()
+    dev = dst / "amk_device.cu"
+    text = dev.read_text()
+    dev.write_text("// an added comment line\n" + text.replace("namespace amk {", "namespace amk {  /* inline */", 1))
+    assert bench._kernel_hash() == h0
+    dev.write_text(text + "\nstatic int amk_hash_probe = 1;\n")
+    assert bench._kernel_hash() != h0
+
+
+def test_traffic_ratio_is_reported_only_for_the_captured_sources():
+    with open(os.path.join(ROOT, "profiles", "decode_kernel_dram_traffic.json")) as f:
+        ent = json.load(f)["workloads"]["llama8b"]
+    t = bench._dram_traffic("llama8b", 1e9)
+    if ent["kernel"] == bench._kernel_hash():
+        assert t == ent["ratio"] * 1e9
+    else:
+        assert t is None
