@@ -38,6 +38,8 @@ CONFIG_SET = [("smollm135m", {}), ("llama1b", {}), ("llama1b", {"weight_dtype": 
               ("llama8b", {"weight_dtype": "bf16"}), ("llama8b_int4", {}), ("llama1b_long4k", {}),
               ("llama1b_long16k", {}), ("llama1b_long32k", {})]
 L2_BYTES = 126e6
+# shapes whose oracle steps the bench also times on the host cores (a bounded sample: about a minute)
+ORACLE_TIMED = ("smollm135m", "llama1b", "llama1b_long4k", "llama1b_long16k", "llama1b_long32k")
 
 
 def metric_for(cfg) -> str:
@@ -441,6 +443,19 @@ def run_gpu(args, cfg, rank, world, local_rank):
                 configs[key] = measure_config(c, peak)
             except Exception as e:  # one shape failing must not hide the headline
                 configs[key] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    if configs is not None and not args.no_cpu_baseline:
+        # the oracle on the host cores, per named shape, over the steps the parity tests compare
+        # (135M all 256, 1B the first 16, long contexts the first 4 per length; the 8B-shaped first 4
+        # are the headline's cpu_baseline)
+        for key in ORACLE_TIMED:
+            if key not in configs or "unavailable" in configs[key]:
+                continue
+            try:
+                tps, secs, sample, cores = oracle_tokens_per_s(_synth.preset(key))
+                configs[key]["cpu_oracle"] = {"tokens_per_s": tps, "ms_per_step": 1000.0 / tps, "cores": cores,
+                                              "sample": sample, "seconds": round(secs, 1)}
+            except Exception as e:  # a reported baseline, never the headline
+                configs[key]["cpu_oracle"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     comparator = None
     if world == 1 and not args.no_comparator:
         try:
